@@ -1,0 +1,296 @@
+/*
+ * oracle.c -- plain, slow CPU oracle for the W8A8 FP8 block-scaled linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link or
+ * call this file: only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark use it.  It shares no code, header, table or constant with the
+ * CUDA library; every value it needs is derived here from the format
+ * definitions.
+ *
+ * What it computes (page "ProCreations/Nanbeige4.3-33B-FP8", introduction and
+ * section "Recipe and calibration"): W8A8 FP8 quantization with E4M3 weights
+ * in 128x128 blocks (standard min-max, data independent) and dynamic
+ * per-token / group-128 activation scales; the linear layer then multiplies
+ * the quantized operands and emits BF16.
+ *
+ * The library specification fixes the details the page leaves open:
+ *   scale = amax / 448 as one IEEE binary32 division (round to nearest even),
+ *   an all-zero group gets scale 1.0,
+ *   code  = E4M3 value nearest to fl32(x / scale), ties to the even mantissa,
+ *           magnitudes above 448 saturate to 448 (never the NaN code),
+ *   the GEMM reference is the FP64 sum over k of the dequantized operands
+ *   (code * scale) -- the order the GPU promotes in is not part of the result's
+ *   definition, only of its rounding.
+ *
+ * Build: gcc -O2 -fopenmp -fno-fast-math -ffp-contract=off -shared -fPIC.
+ * x86-64 evaluates float expressions in binary32 (FLT_EVAL_METHOD 0) and keeps
+ * subnormals unless fast-math flags are given, so every float operation below
+ * is the IEEE operation it reads as.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define GROUP 128 /* channels per activation group; rows and cols of a weight block */
+
+/* BF16 is the upper half of a binary32 pattern, so widening is exact. */
+static float bf16_bits_to_float(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/*
+ * E4M3 "fn" format (OCP 8-bit floating point, the variant the page names
+ * "e4m3fn"): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no
+ * infinities, and S.1111.111 reserved for NaN.  Normal values are
+ * (1 + m/8) * 2^(e-7) for e = 1..15 (e = 15 only for m <= 6, so the largest is
+ * 1.75 * 2^8 = 448); subnormals are (m/8) * 2^-6.
+ */
+double oracle_e4m3_decode(uint8_t code)
+{
+    int sign = code >> 7;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ((double)m / 8.0) * ldexp(1.0, -6);
+    else
+        v = (1.0 + (double)m / 8.0) * ldexp(1.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Round a non-negative real (held exactly in a double) to the nearest integer,
+ * ties to the even integer. */
+static double round_half_even(double n)
+{
+    double lo = floor(n);
+    double frac = n - lo; /* exact: n has at most 53 significant bits */
+    if (frac > 0.5)
+        return lo + 1.0;
+    if (frac < 0.5)
+        return lo;
+    return (fmod(lo, 2.0) == 0.0) ? lo : lo + 1.0;
+}
+
+/* Bit pattern of a non-negative value that is exactly an E4M3 value <= 448. */
+static uint8_t e4m3_bits_of_exact(double v)
+{
+    int E;
+    if (v == 0.0)
+        return 0;
+    (void)frexp(v, &E);   /* v = f * 2^E, f in [0.5, 1) */
+    int e = E - 1;        /* floor(log2 v) */
+    if (e < -6) {         /* subnormal: v = m * 2^-9 */
+        int m = (int)(v / ldexp(1.0, -9));
+        return (uint8_t)m;
+    }
+    int m = (int)(v / ldexp(1.0, e - 3)) - 8; /* v = (8 + m) * 2^(e-3) */
+    return (uint8_t)(((e + 7) << 3) | m);
+}
+
+/*
+ * Encode a finite binary32 value: round to the nearest point of the E4M3 grid
+ * (ties to even mantissa), then saturate magnitudes above 448 to 448.
+ * Within the binade [2^e, 2^(e+1)) the grid spacing is 2^(e-3); below 2^-6
+ * (the subnormal range) it stays 2^-9.  The sign is kept, so -0 gives 0x80.
+ */
+uint8_t oracle_e4m3_encode(float y)
+{
+    uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    double a = fabs((double)y);
+    if (a == 0.0)
+        return sign;
+    int E;
+    (void)frexp(a, &E);
+    int e = E - 1;
+    if (e < -6)
+        e = -6;
+    double quantum = ldexp(1.0, e - 3);
+    double n = a / quantum;                 /* exact: division by a power of two */
+    double v = round_half_even(n) * quantum; /* may round up into the next binade */
+    if (v > 448.0)
+        v = 448.0;
+    return sign | e4m3_bits_of_exact(v);
+}
+
+void oracle_e4m3_encode_array(const float *y, int64_t n, uint8_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; i++)
+        out[i] = oracle_e4m3_encode(y[i]);
+}
+
+void oracle_e4m3_decode_array(const uint8_t *c, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = oracle_e4m3_decode(c[i]);
+}
+
+/* scale of a group or block from its amax: amax / 448 in binary32, or 1 for zero */
+static float scale_from_amax(float amax)
+{
+    if (amax == 0.0f)
+        return 1.0f;
+    return amax / 448.0f;
+}
+
+/*
+ * Dynamic per-token, group-128 activation quantization.
+ * x: BF16 bit patterns [M, K] row-major; q: E4M3 codes [M, K]; s: FP32 [M, K/128].
+ * Group g of row m is channels [128 g, 128 g + 128) of that row.
+ */
+void oracle_quantize_act(const uint16_t *x, int64_t M, int64_t K, uint8_t *q, float *s)
+{
+    int64_t G = K / GROUP;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t g = 0; g < G; g++) {
+            const uint16_t *xg = x + m * K + g * GROUP;
+            float amax = 0.0f;
+            for (int i = 0; i < GROUP; i++) {
+                float a = fabsf(bf16_bits_to_float(xg[i]));
+                if (a > amax)
+                    amax = a;
+            }
+            float sc = scale_from_amax(amax);
+            s[m * G + g] = sc;
+            for (int i = 0; i < GROUP; i++) {
+                float y = bf16_bits_to_float(xg[i]) / sc;
+                q[m * K + g * GROUP + i] = oracle_e4m3_encode(y);
+            }
+        }
+    }
+}
+
+/*
+ * Same as oracle_quantize_act, restricted to the listed rows.  Output row r of
+ * q / s holds input row rows[r].
+ */
+void oracle_quantize_act_rows(const uint16_t *x, int64_t M, int64_t K, const int64_t *rows,
+                              int64_t nrows, uint8_t *q, float *s)
+{
+    int64_t G = K / GROUP;
+    (void)M;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < nrows; r++)
+        oracle_quantize_act(x + rows[r] * K, 1, K, q + r * K, s + r * G);
+}
+
+/*
+ * Offline 128x128 block min-max weight quantization.
+ * w: BF16 bit patterns [N, K] (out x in, row-major); q: E4M3 [N, K];
+ * s: FP32 [N/128, K/128].  Block (i, j) is rows [128 i, +128) x cols [128 j, +128).
+ */
+void oracle_quantize_weight(const uint16_t *w, int64_t N, int64_t K, uint8_t *q, float *s)
+{
+    int64_t NB = N / GROUP, KB = K / GROUP;
+#pragma omp parallel for schedule(static) collapse(2)
+    for (int64_t bi = 0; bi < NB; bi++) {
+        for (int64_t bj = 0; bj < KB; bj++) {
+            float amax = 0.0f;
+            for (int r = 0; r < GROUP; r++)
+                for (int c = 0; c < GROUP; c++) {
+                    float a = fabsf(bf16_bits_to_float(w[(bi * GROUP + r) * K + bj * GROUP + c]));
+                    if (a > amax)
+                        amax = a;
+                }
+            float sc = scale_from_amax(amax);
+            s[bi * KB + bj] = sc;
+            for (int r = 0; r < GROUP; r++)
+                for (int c = 0; c < GROUP; c++) {
+                    int64_t idx = (bi * GROUP + r) * K + bj * GROUP + c;
+                    q[idx] = oracle_e4m3_encode(bf16_bits_to_float(w[idx]) / sc);
+                }
+        }
+    }
+}
+
+/*
+ * FP64 reference of the block-scaled GEMM, Y = A * W^T with
+ *   A[m, k] = decode(qa[m, k]) * sa[m, k/128]
+ *   W[n, k] = decode(qw[n, k]) * sw[n/128, k/128]
+ * and out[r, n] = sum over k = 0..K-1 (ascending) of A[rows[r], k] * W[n, k],
+ * accumulated in double.  Only the listed rows of A are evaluated, so large
+ * shapes can be checked on a sample; pass rows = 0..M-1 for all of them.
+ * qa / sa are indexed by the original row number.
+ */
+void oracle_gemm_ref(const uint8_t *qa, const float *sa, const uint8_t *qw, const float *sw,
+                     int64_t M, int64_t N, int64_t K, const int64_t *rows, int64_t nrows,
+                     double *out)
+{
+    int64_t KB = K / GROUP;
+    const int64_t NCHUNK = 128;
+    (void)M;
+    double *arows = (double *)malloc(sizeof(double) * (size_t)(nrows * K));
+    double *wrows = (double *)malloc(sizeof(double) * (size_t)(NCHUNK * K));
+    if (!arows || !wrows) {
+        free(arows);
+        free(wrows);
+        for (int64_t i = 0; i < nrows * N; i++)
+            out[i] = NAN;
+        return;
+    }
+    /* dequantize the requested activation rows once */
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < nrows; r++) {
+        int64_t m = rows[r];
+        for (int64_t k = 0; k < K; k++)
+            arows[r * K + k] = oracle_e4m3_decode(qa[m * K + k]) * (double)sa[m * KB + k / GROUP];
+    }
+    for (int64_t n0 = 0; n0 < N; n0 += NCHUNK) {
+        int64_t nc = (N - n0 < NCHUNK) ? (N - n0) : NCHUNK;
+        /* dequantize a chunk of weight rows */
+#pragma omp parallel for schedule(static)
+        for (int64_t j = 0; j < nc; j++) {
+            int64_t n = n0 + j;
+            for (int64_t k = 0; k < K; k++)
+                wrows[j * K + k] =
+                    oracle_e4m3_decode(qw[n * K + k]) * (double)sw[(n / GROUP) * KB + k / GROUP];
+        }
+        /* plain dot products */
+#pragma omp parallel for schedule(static)
+        for (int64_t r = 0; r < nrows; r++) {
+            const double *a = arows + r * K;
+            for (int64_t j = 0; j < nc; j++) {
+                const double *w = wrows + j * K;
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; k++)
+                    acc += a[k] * w[k];
+                out[r * N + n0 + j] = acc;
+            }
+        }
+    }
+    free(arows);
+    free(wrows);
+}
+
+/* BF16 rounding of a double, nearest-even on the BF16 grid (8 significant bits),
+ * through binary32 first only when that is exact; used to express the
+ * closed-form expectations of the exact-arithmetic tests. */
+uint16_t oracle_bf16_round(double v)
+{
+    /* Decompose v exactly and round its significand to 8 bits, ties to even. */
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    int E;
+    (void)frexp(a, &E);
+    int e = E - 1;                 /* floor(log2 a) */
+    if (e < -126)
+        e = -126;                  /* BF16 subnormals share the smallest normal quantum */
+    double quantum = ldexp(1.0, e - 7);
+    double r = round_half_even(a / quantum) * quantum;
+    if (r >= ldexp(1.0, 128))
+        return sign | 0x7F80;      /* overflow to infinity */
+    float f = (float)r;            /* exact: r has <= 8 significant bits in range */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFF));
+}

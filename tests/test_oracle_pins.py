@@ -1,0 +1,349 @@
+"""Pins of the CPU oracle against facts fixed outside it.
+
+Each check is chosen so that a plausible slip in the oracle fails it:
+
+* E4M3 decode: torch's float8_e4m3fn decoding of all 256 codes, plus the
+  landmark values of the format (448 max, 2^-9 smallest subnormal, NaN code).
+* E4M3 encode: exhaustive nearest-value brute force over every binary32 bit
+  pattern whose magnitude lies in [2^-24, 1024) (ties to the even mantissa,
+  saturation), and torch's clamp + RNE cast over all 2^32 finite patterns.
+* Quantizers: the min-max invariants (max element codes to +-448; the scale
+  is fl32(amax/448) and 448 s is within 2^-24 amax of amax; codes within
+  +-448, never NaN; an all-zero group has scale 1 and zero codes; identity on
+  E4M3-representable groups whose amax is 448 * 2^j), each code equal to
+  torch's cast of the binary32 quotient, and block/group placement checked
+  with blocks of distinct amax (a transposed or shifted index fails).
+* GEMM: exact rational sums (Python integers) on several tile-spanning
+  shapes, including the 128x128x128 brute force, with the FP64 summation
+  error bound; identity and permuted one-hot weights in closed form; an
+  exact-arithmetic regime where FP64 must be exact; M = 1 as numpy's dot.
+* BF16 rounding: torch's RNE cast on binary32-representable values.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact
+import oracle
+import workloads
+
+pytestmark = pytest.mark.usefixtures("oracle_lib")
+
+
+def bf16(a) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------------------- E4M3 format
+
+def test_decode_matches_torch_on_all_codes():
+    got = oracle.e4m3_decode(np.arange(256, dtype=np.uint8))
+    ref = exact.E4M3
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert nan.sum() == 2 and nan[0x7F] and nan[0xFF]
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_decode_landmarks():
+    d = oracle.e4m3_decode(np.array([0x00, 0x01, 0x07, 0x08, 0x38, 0x7E, 0x80, 0xFE], np.uint8))
+    assert d[0] == 0.0 and d[1] == 2.0 ** -9 and d[2] == 7 * 2.0 ** -9
+    assert d[3] == 2.0 ** -6 and d[4] == 1.0 and d[5] == 448.0
+    assert d[6] == 0.0 and math.copysign(1.0, d[6]) == -1.0 and d[7] == -448.0
+
+
+def _brute_force_encode(y: np.ndarray) -> np.ndarray:
+    """Nearest finite E4M3 value (ties: even mantissa = even code), saturating at 448."""
+    vals = exact.E4M3[:0x7F]                    # the 127 non-negative finite values, ascending
+    a = np.abs(y.astype(np.float64))
+    hi = np.searchsorted(vals, a, side="left")  # first value >= a
+    hi = np.minimum(hi, vals.size - 1)
+    lo = np.maximum(hi - 1, 0)
+    dlo = a - vals[lo]
+    dhi = vals[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(a >= vals[-1], 0x7E, code)  # everything above the largest value saturates
+    code = np.where(a <= vals[0], 0, code)
+    sign = np.signbit(y).astype(np.uint8) << 7
+    return (code.astype(np.uint8) | sign)
+
+
+def test_encode_brute_force_exhaustive_range():
+    # every positive binary32 pattern with magnitude in [2^-24, 2^10), and its negation on
+    # a strided subset; below 2^-24 everything is 0 (checked on a sample in the next test)
+    lo = np.float32(2.0 ** -24).view(np.uint32)
+    hi = np.float32(1024.0).view(np.uint32)
+    step = 1 << 24
+    for start in range(int(lo), int(hi), step):
+        pat = np.arange(start, min(start + step, int(hi)), dtype=np.uint32)
+        y = pat.view(np.float32)
+        got = oracle.e4m3_encode(y)
+        ref = _brute_force_encode(y)
+        bad = np.nonzero(got != ref)[0]
+        assert bad.size == 0, (y[bad[:5]], got[bad[:5]], ref[bad[:5]])
+        yn = -y[::97]
+        assert np.array_equal(oracle.e4m3_encode(yn), _brute_force_encode(yn))
+
+
+def test_encode_matches_torch_on_all_finite_patterns():
+    step = 1 << 26
+    for start in range(0, 1 << 32, step):
+        pat = np.arange(start, start + step, dtype=np.uint64).astype(np.uint32)
+        y = pat.view(np.float32)
+        y = y[np.isfinite(y)]
+        got = oracle.e4m3_encode(y)
+        ref = exact.torch_encode(y)
+        bad = np.nonzero(got != ref)[0]
+        assert bad.size == 0, (y[bad[:5]], got[bad[:5]], ref[bad[:5]])
+
+
+def test_encode_landmarks():
+    y = np.array([448.0, 463.99, 464.0, 464.01, 1e30, 2.0 ** -10, 3 * 2.0 ** -11, -0.0,
+                  0.3, 2.0 ** -6 - 2.0 ** -11, 240.0, 232.0, 248.0], dtype=np.float32)
+    got = oracle.e4m3_encode(y)
+    # 464 is the midpoint between 448 (mantissa 110) and 480 (not finite): ties to even -> 448
+    assert list(got[:5]) == [0x7E] * 5
+    assert got[5] == 0x00                        # 2^-10: tie between 0 and 2^-9 -> even (0)
+    assert got[6] == 0x01                        # 0.75 * 2^-9 rounds to 2^-9
+    assert got[7] == 0x80                        # sign of zero kept
+    assert exact.dq(got[8]) == 0.3125
+    assert got[9] == 0x08                        # rounds up out of the subnormal range
+    assert exact.dq(got[10]) == 240.0
+    assert exact.dq(got[11]) == 224.0            # 232 ties 224 (even) / 240 (odd)
+    assert exact.dq(got[12]) == 256.0            # 248 ties 240 (odd) / 256 (even)
+
+
+# ----------------------------------------------------------------------------- quantizers
+
+def _group_view(x: np.ndarray) -> np.ndarray:
+    M, K = x.shape
+    return x.reshape(M, K // 128, 128)
+
+
+def _check_minmax_invariants(xf: np.ndarray, q: np.ndarray, s: np.ndarray):
+    """xf: [..., 128] groups in float32; q: codes of the same shape; s: [...] scales."""
+    amax = np.abs(xf).max(axis=-1)
+    zero = amax == 0
+    assert not np.any((q & 0x7F) == 0x7F), "NaN code produced"
+    assert np.all(np.abs(exact.dq(q)) <= 448.0)
+    # scale is one binary32 division of amax by 448 (numpy float32 division is IEEE RN)
+    expect = np.where(zero, np.float32(1.0), (amax / np.float32(448.0)).astype(np.float32))
+    assert np.array_equal(s.view(np.uint32), expect.astype(np.float32).view(np.uint32))
+    nz = ~zero
+    err = np.abs(448.0 * s[nz].astype(np.float64) - amax[nz].astype(np.float64))
+    # half an ulp of s, relative for normal scales and 2^-150 absolute for subnormal ones
+    assert np.all(err <= np.maximum(2.0 ** -24 * amax[nz].astype(np.float64), 448.0 * 2.0 ** -150))
+    # the max element(s) of every non-zero group code to +-448
+    is_max = (np.abs(xf) == amax[..., None]) & nz[..., None]
+    assert np.all((q[is_max] & 0x7F) == 0x7E)
+    # all-zero groups: scale 1 and signed zero codes
+    assert np.all((q[zero] & 0x7F) == 0)
+    # each code is torch's saturating RNE cast of the binary32 quotient
+    quot = (xf / s[..., None]).astype(np.float32)
+    assert np.array_equal(q, exact.torch_encode(quot))
+
+
+@pytest.mark.parametrize("M,K,kind", [(1, 128, "normal"), (5, 384, "normal"),
+                                      (16, 7168, "kproj"), (33, 1024, "t3"), (8, 512, "tiny")])
+def test_quantize_act_invariants(M, K, kind):
+    if kind == "kproj":
+        x = workloads.KPROJ_M16.make_x()
+    elif kind == "t3":
+        x = workloads.activation(M, K, 77, t3_channels=10, outliers=3)
+    elif kind == "tiny":
+        # BF16 subnormal magnitudes: scales become subnormal binary32 values
+        rng = np.random.default_rng(5)
+        x = bf16(rng.standard_normal((M, K)).astype(np.float32) * np.float32(1e-39))
+    else:
+        x = workloads.activation(M, K, 11 + M)
+    q, s = oracle.quantize_act(x)
+    xf = x.float().numpy()
+    _check_minmax_invariants(_group_view(xf), _group_view(q), s)
+    if kind == "tiny":
+        assert np.any((s > 0) & (s < np.finfo(np.float32).tiny)), "no subnormal scale exercised"
+
+
+def test_quantize_act_zero_row_and_negative_zero():
+    x = np.zeros((2, 256), dtype=np.float32)
+    x[1, :128] = -0.0
+    x[1, 128:] = np.linspace(-3, 3, 128)
+    q, s = oracle.quantize_act(bf16(x))
+    assert np.all(s[0] == 1.0) and np.all(q[0] == 0x00)
+    assert s[1, 0] == 1.0 and np.all(q[1, :128] == 0x80)
+    assert s[1, 1] == np.float32(3.0) / np.float32(448.0)
+
+
+def test_quantize_act_identity_on_representable_groups():
+    # every group holds E4M3 values (times 2^j) with amax exactly 448 * 2^j: codes reproduce x
+    rng = np.random.default_rng(3)
+    finite = np.array([c for c in range(0x7F)], dtype=np.uint8)
+    M, G = 6, 4
+    codes = rng.choice(finite, size=(M, G, 128))
+    codes[:, :, 0] = 0x7E
+    signs = rng.integers(0, 2, size=codes.shape).astype(np.uint8) << 7
+    codes = codes | signs
+    j = rng.integers(-20, 20, size=(M, G))
+    xf = exact.dq(codes) * np.ldexp(1.0, j)[..., None]
+    x = bf16(xf.reshape(M, G * 128))               # E4M3 values fit BF16 exactly
+    assert np.array_equal(x.double().numpy(), xf.reshape(M, G * 128))
+    q, s = oracle.quantize_act(x)
+    assert np.array_equal(s, np.ldexp(np.float32(1.0), j).astype(np.float32))
+    assert np.array_equal(exact.dq(q), exact.dq(codes.reshape(M, G * 128)))
+
+
+def test_quantize_act_every_bf16_of_a_binade():
+    # one group per binade: the 128 BF16 values 2^e * (1 + i/128), i = 0..127
+    rows = []
+    for e in (-130, -20, -1, 0, 7, 100):
+        rows.append(np.ldexp(1.0 + np.arange(128) / 128.0, e))
+    x = bf16(np.array(rows))
+    q, s = oracle.quantize_act(x)
+    _check_minmax_invariants(_group_view(x.float().numpy()), _group_view(q), s)
+
+
+def test_quantize_act_group_placement():
+    # group g of row m has amax 2^(m - g): a transposed or shifted group index changes s
+    M, G = 3, 5
+    x = np.zeros((M, G * 128), dtype=np.float32)
+    for m in range(M):
+        for g in range(G):
+            x[m, g * 128 + (7 * g + m) % 128] = 2.0 ** (m - g)
+    q, s = oracle.quantize_act(bf16(x))
+    for m in range(M):
+        for g in range(G):
+            assert s[m, g] == np.float32(2.0 ** (m - g)) / np.float32(448.0)
+
+
+def test_quantize_weight_invariants_and_placement():
+    N, K = 384, 512
+    w = workloads.weight(N, K, 42).float().numpy()
+    # give block (i, j) amax-scale 2^(i - 2 j) so placement errors change the scales
+    for i in range(N // 128):
+        for j in range(K // 128):
+            w[i * 128:(i + 1) * 128, j * 128:(j + 1) * 128] *= 2.0 ** (i - 2 * j)
+    w[128:256, 0:128] = 0.0                        # one all-zero block
+    wt = bf16(w)
+    q, s = oracle.quantize_weight(wt)
+    wf = wt.float().numpy()
+    blocks = wf.reshape(N // 128, 128, K // 128, 128).transpose(0, 2, 1, 3).reshape(
+        N // 128, K // 128, 128 * 128)
+    qb = q.reshape(N // 128, 128, K // 128, 128).transpose(0, 2, 1, 3).reshape(
+        N // 128, K // 128, 128 * 128)
+    _check_minmax_invariants(blocks, qb, s)
+    assert s[1, 0] == 1.0
+
+
+def test_quantize_weight_identity():
+    # identity weight: every diagonal block has amax 1, codes 448 on the diagonal
+    w = bf16(np.eye(256, dtype=np.float32))
+    q, s = oracle.quantize_weight(w)
+    assert np.all(s[[0, 1], [0, 1]] == np.float32(1.0) / np.float32(448.0))
+    assert np.all(s[[0, 1], [1, 0]] == 1.0)
+    assert np.array_equal(q, np.where(np.eye(256, dtype=bool), 0x7E, 0).astype(np.uint8))
+
+
+# ----------------------------------------------------------------------------- GEMM reference
+
+def _random_operands(M, N, K, seed):
+    x = workloads.activation(M, K, seed, outliers=2)
+    w = workloads.weight(N, K, seed + 1)
+    qa, sa = oracle.quantize_act(x)
+    qw, sw = oracle.quantize_weight(w)
+    return qa, sa, qw, sw
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (3, 256, 384), (1, 128, 1024)])
+def test_gemm_exact_rational(M, N, K):
+    qa, sa, qw, sw = _random_operands(M, N, K, 100 + M)
+    got = oracle.gemm_ref(qa, sa, qw, sw)
+    ex, abs_sum = exact.exact_gemm(qa, sa, qw, sw)
+    exf = np.array([[float(v) for v in row] for row in ex])
+    # recursive FP64 summation of K exact-in-FP64? products: |err| <= (K+1) u sum|terms|
+    bound = (K + 1) * 2.0 ** -53 * abs_sum * (1 + 1e-9)
+    assert np.all(np.abs(got - exf) <= bound + np.abs(exf) * 2.0 ** -53)
+
+
+def test_gemm_exact_arithmetic_regime():
+    # small-integer codes and power-of-two scales: every partial sum is exact in FP64
+    rng = np.random.default_rng(9)
+    M, N, K = 7, 256, 512
+    small = np.array([0x00, 0x38, 0x40, 0x44, 0x48, 0x4A, 0xB8, 0xC0, 0xC4], np.uint8)  # 0,1,2,3,4,5,-1,-2,-3
+    qa = rng.choice(small, size=(M, K))
+    qw = rng.choice(small, size=(N, K))
+    sa = np.ldexp(np.float32(1.0), rng.integers(-6, 6, size=(M, K // 128))).astype(np.float32)
+    sw = np.ldexp(np.float32(1.0), rng.integers(-6, 6, size=(N // 128, K // 128))).astype(np.float32)
+    got = oracle.gemm_ref(qa, sa, qw, sw)
+    ex, _ = exact.exact_gemm(qa, sa, qw, sw)
+    assert all(float(ex[i, j]) == got[i, j] and ex[i, j] == got[i, j]
+               for i in range(M) for j in range(N))
+
+
+def test_gemm_identity_weight_closed_form():
+    M = 9
+    x = workloads.activation(M, 128, 21, outliers=1)
+    qa, sa = oracle.quantize_act(x)
+    qw, sw = oracle.quantize_weight(bf16(np.eye(128, dtype=np.float32)))
+    got = oracle.gemm_ref(qa, sa, qw, sw)
+    # Y[m, n] = dq(qa[m, n]) sa[m, 0] * 448 * sw, one exact product per output
+    closed = exact.dq(qa) * sa[:, :1].astype(np.float64) * 448.0 * np.float64(sw[0, 0])
+    assert np.array_equal(got, closed)
+
+
+def test_gemm_permuted_one_hot_closed_form():
+    # W[n, pi(n)] = 1: Y[m, n] = A[m, pi(n)] * 448 * sw[n/128, pi(n)/128]; catches transposition
+    M, N, K = 5, 256, 384
+    rng = np.random.default_rng(4)
+    pi = rng.permutation(K)[:N]
+    w = np.zeros((N, K), dtype=np.float32)
+    w[np.arange(N), pi] = 1.0
+    x = workloads.activation(M, K, 31)
+    qa, sa = oracle.quantize_act(x)
+    qw, sw = oracle.quantize_weight(bf16(w))
+    got = oracle.gemm_ref(qa, sa, qw, sw)
+    a = exact.dq(qa) * np.repeat(sa.astype(np.float64), 128, axis=1)
+    closed = a[:, pi] * 448.0 * sw[np.arange(N) // 128, pi // 128].astype(np.float64)[None, :]
+    assert np.array_equal(got, closed)
+
+
+def test_gemm_single_row_is_a_dot_product():
+    qa, sa, qw, sw = _random_operands(1, 128, 896, 7)
+    a = exact.dq(qa[0]) * np.repeat(sa[0].astype(np.float64), 128)
+    got = oracle.gemm_ref(qa, sa, qw, sw)[0]
+    for n in (0, 63, 127):
+        w = exact.dq(qw[n]) * np.repeat(sw[n // 128].astype(np.float64), 128)
+        assert abs(got[n] - np.dot(a, w)) <= 1e-12 * np.abs(a * w).sum()
+
+
+def test_gemm_row_subset_matches_full():
+    qa, sa, qw, sw = _random_operands(40, 256, 256, 12)
+    full = oracle.gemm_ref(qa, sa, qw, sw)
+    rows = np.array([39, 0, 17, 17], dtype=np.int64)
+    assert np.array_equal(oracle.gemm_ref(qa, sa, qw, sw, rows=rows), full[rows])
+
+
+def test_linear_ref_composes_quantize_and_gemm():
+    x = workloads.activation(12, 384, 5, outliers=2)
+    qw, sw = oracle.quantize_weight(workloads.weight(128, 384, 6))
+    qa, sa = oracle.quantize_act(x)
+    rows = np.array([3, 11], dtype=np.int64)
+    assert np.array_equal(oracle.linear_ref(x, qw, sw, rows=rows),
+                          oracle.gemm_ref(qa, sa, qw, sw, rows=rows))
+
+
+# ----------------------------------------------------------------------------- BF16 rounding
+
+def test_bf16_round_matches_torch_on_float32_values():
+    rng = np.random.default_rng(1)
+    v = np.concatenate([rng.standard_normal(4000).astype(np.float32) * 100,
+                        np.float32([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -0.0,
+                                    3e38, 1e-40, -2.5e-39])])
+    ref = bits(torch.from_numpy(v).to(torch.bfloat16))
+    got = oracle.bf16_round(v.astype(np.float64))
+    assert np.array_equal(got, ref)
