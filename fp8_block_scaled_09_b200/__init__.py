@@ -1,0 +1,198 @@
+"""W8A8 FP8 block-scaled linear layer for B200 (sm_100a).
+
+Python binding of the C ABI in ``include/fp8bq.h`` (library ``libfp8bq.so``
+built in this directory by ``build.py``).  This module only marshals torch
+tensors (device memory and the current CUDA stream) into the C calls; every
+step of the computation runs in the library's CUDA kernels.  There is no CPU
+fallback: if the library is missing or no sm_100 device is current, the calls
+raise.
+
+Functions (names follow the C ABI without the ``fp8bq_`` prefix):
+
+* ``quantize_act(x)``        BF16 [M, K] -> (E4M3 codes uint8 [M, K], FP32 [M, K/128])
+* ``quantize_weight(w)``     BF16 [N, K] -> (E4M3 codes uint8 [N, K], FP32 [N/128, K/128])
+* ``gemm(qa, sa, qw, sw)``   -> BF16 [M, N]
+* ``linear(x, qw, sw)``      -> BF16 [M, N], activation quantization fused into the call
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "Fp8bqError", "lib", "quantize_act", "quantize_weight", "gemm", "linear",
+    "workspace_size", "new_workspace", "workspace_init", "last_device_status",
+    "launch_count", "status_string", "OP_GEMM", "OP_LINEAR", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bq.so")
+OP_GEMM = 0
+OP_LINEAR = 1
+
+STATUS_NAMES = {
+    0: "FP8BQ_OK", 1: "FP8BQ_ERR_INVALID_ARG", 2: "FP8BQ_ERR_UNSUPPORTED_SHAPE",
+    3: "FP8BQ_ERR_MISALIGNED", 4: "FP8BQ_ERR_WORKSPACE", 5: "FP8BQ_ERR_CUDA",
+    6: "FP8BQ_ERR_TIMEOUT", 7: "FP8BQ_ERR_NO_DEVICE",
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class Fp8bqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libfp8bq.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m fp8_block_scaled_09_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+        st = ctypes.c_int
+        L.fp8bq_quantize_act.argtypes = [P, I, I, P, P, P]
+        L.fp8bq_quantize_weight.argtypes = [P, I, I, P, P, P]
+        L.fp8bq_gemm.argtypes = [P, P, P, P, I, I, I, P, P, S, P]
+        L.fp8bq_linear.argtypes = [P, P, P, I, I, I, P, P, S, P]
+        L.fp8bq_workspace_size.argtypes = [ctypes.c_int, I, I, I]
+        L.fp8bq_workspace_size.restype = S
+        L.fp8bq_workspace_init.argtypes = [P, S, P]
+        L.fp8bq_last_device_status.argtypes = [P]
+        L.fp8bq_status_string.argtypes = [st]
+        L.fp8bq_status_string.restype = ctypes.c_char_p
+        L.fp8bq_launch_count.argtypes = []
+        L.fp8bq_launch_count.restype = ctypes.c_uint64
+        L.fp8bq_version.argtypes = []
+        L.fp8bq_version.restype = ctypes.c_int
+        for name in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
+                     "fp8bq_workspace_init", "fp8bq_last_device_status"):
+            getattr(L, name).restype = st
+        _lib = L
+        return L
+
+
+def status_string(status: int) -> str:
+    return lib().fp8bq_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise Fp8bqError(status, what)
+
+
+def _stream(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _codes(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8)
+    if t.dtype != torch.uint8:
+        raise TypeError(f"E4M3 codes must be uint8 or float8_e4m3fn, got {t.dtype}")
+    return t
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+
+
+def workspace_size(op: int, M: int, N: int, K: int) -> int:
+    return int(lib().fp8bq_workspace_size(op, M, N, K))
+
+
+def new_workspace(op: int, M: int, N: int, K: int, device) -> torch.Tensor:
+    """A zero-filled (initial-state) workspace for this operation and shape."""
+    return torch.zeros(max(workspace_size(op, M, N, K), 256), dtype=torch.uint8, device=device)
+
+
+def workspace_init(ws: torch.Tensor) -> None:
+    _check(lib().fp8bq_workspace_init(_ptr(ws), ws.numel(), _stream(ws)), "fp8bq_workspace_init")
+
+
+def quantize_act(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if s is None:
+        s = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+    _check(lib().fp8bq_quantize_act(_ptr(x), M, K, _ptr(q), _ptr(s), _stream(x)),
+           "fp8bq_quantize_act")
+    return q, s
+
+
+def quantize_weight(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None):
+    _need(w, torch.bfloat16, "w")
+    N, K = w.shape
+    if q is None:
+        q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    if s is None:
+        s = torch.empty((N // 128, K // 128), dtype=torch.float32, device=w.device)
+    _check(lib().fp8bq_quantize_weight(_ptr(w), N, K, _ptr(q), _ptr(s), _stream(w)),
+           "fp8bq_quantize_weight")
+    return q, s
+
+
+def gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+         out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    qa, qw = _codes(qa), _codes(qw)
+    _need(qa, torch.uint8, "qa")
+    _need(qw, torch.uint8, "qw")
+    _need(sa, torch.float32, "sa")
+    _need(sw, torch.float32, "sw")
+    M, K = qa.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.device)
+    if workspace is None:
+        workspace = new_workspace(OP_GEMM, M, N, K, qa.device)
+    _check(lib().fp8bq_gemm(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), M, N, K, _ptr(out),
+                            _ptr(workspace), workspace.numel(), _stream(qa)), "fp8bq_gemm")
+    return out
+
+
+def linear(x: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, out: torch.Tensor | None = None,
+           workspace: torch.Tensor | None = None) -> torch.Tensor:
+    qw = _codes(qw)
+    _need(x, torch.bfloat16, "x")
+    _need(qw, torch.uint8, "qw")
+    _need(sw, torch.float32, "sw")
+    M, K = x.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = new_workspace(OP_LINEAR, M, N, K, x.device)
+    _check(lib().fp8bq_linear(_ptr(x), _ptr(qw), _ptr(sw), M, N, K, _ptr(out), _ptr(workspace),
+                              workspace.numel(), _stream(x)), "fp8bq_linear")
+    return out
+
+
+def last_device_status(device=None) -> int:
+    """Synchronizes the current stream and returns/clears the device status word."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    return int(lib().fp8bq_last_device_status(s))
+
+
+def launch_count() -> int:
+    return int(lib().fp8bq_launch_count())

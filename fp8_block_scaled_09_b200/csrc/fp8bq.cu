@@ -1,0 +1,326 @@
+// fp8bq.cu -- the C ABI declared in include/fp8bq.h: host-side argument
+// validation, per-device set-up, TMA descriptor encoding and kernel dispatch.
+//
+// All kernels live in this one translation unit so the device status word is a
+// single per-device symbol.  Dispatch:
+//   quantize_act     -> quantize_act_kernel (HBM-bound, grid = k x SMs)
+//   quantize_weight  -> quantize_weight_kernel (one CTA per 128x128 block)
+//   gemm, M <= 16    -> decode::gemm_decode_kernel (stream-K over weight blocks)
+//   gemm, M > 16     -> prefill::gemm_prefill_kernel<256> (persistent tcgen05)
+//   linear           -> quantize_act into the workspace, then the gemm path
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "fp8bq.h"
+#include "gemm_decode.cuh"
+#include "gemm_prefill.cuh"
+#include "ptx.cuh"
+#include "quantize.cuh"
+
+namespace fp8bq {
+
+// Per-device status word: FP8BQ_OK or FP8BQ_ERR_TIMEOUT (set by a kernel that
+// abandoned a wait).  Read and cleared by fp8bq_last_device_status().
+__device__ int g_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kPrefillBN = 256;
+constexpr int64_t kDecodeMaxM = decode::MT;
+
+std::atomic<uint64_t> g_launches{0};
+
+struct DeviceInfo {
+    int sm_count = 0;
+    int *status = nullptr;  // device address of g_status
+    bool supported = false;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+EncodeTiledFn encode_fn() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    return g_encode;
+}
+
+// Current device's info, set up once per device (kernel attributes, status word).
+const DeviceInfo *device_info() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::call_once(g_dev_once[dev], [dev] {
+        DeviceInfo &d = g_dev[dev];
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return;
+        if (major != 10 || minor != 0) return;  // built for sm_100a only
+        if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), g_status) != cudaSuccess)
+            return;
+        if (cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess) return;
+        if (cudaFuncSetAttribute(prefill::gemm_prefill_kernel<kPrefillBN>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 prefill::Layout<kPrefillBN>::kDynamicSmem) != cudaSuccess)
+            return;
+        if (cudaFuncSetAttribute(decode::gemm_decode_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::Layout::kDynamicSmem) != cudaSuccess)
+            return;
+        if (cudaDeviceSynchronize() != cudaSuccess) return;
+        d.supported = true;
+    });
+    const DeviceInfo *d = &g_dev[dev];
+    return d->supported ? d : nullptr;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxDim = 0x7FFFFFFF;
+constexpr int64_t kMaxBytes = int64_t(1) << 40;
+
+fp8bq_status check_mk(int64_t M, int64_t K) {
+    if (M < 0 || K <= 0) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    if (K % 128 != 0 || M > kMaxDim || K > kMaxDim) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    if (M > 0 && K > kMaxBytes / 2 / M) return FP8BQ_ERR_UNSUPPORTED_SHAPE;  // BF16 [M, K]
+    return FP8BQ_OK;
+}
+
+fp8bq_status check_mnk(int64_t M, int64_t N, int64_t K) {
+    fp8bq_status st = check_mk(M, K);
+    if (st != FP8BQ_OK) return st;
+    if (N <= 0 || N % 128 != 0 || N > kMaxDim) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    if (N > kMaxBytes / K) return FP8BQ_ERR_UNSUPPORTED_SHAPE;             // codes [N, K]
+    if (M > 0 && N > kMaxBytes / 2 / M) return FP8BQ_ERR_UNSUPPORTED_SHAPE;  // BF16 [M, N]
+    return FP8BQ_OK;
+}
+
+fp8bq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FP8BQ_OK : FP8BQ_ERR_CUDA; }
+
+// 2-D uint8 tensor map over a row-major [rows, cols] byte matrix, box
+// [box_rows, 128 bytes], 128-byte swizzle, zero fill out of bounds.
+bool make_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+    const cuuint32_t box[2] = {128u, box_rows};
+    const cuuint32_t elem[2] = {1u, 1u};
+    std::memset(map, 0, sizeof(*map));
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box,
+               elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t round256(int64_t b) { return static_cast<size_t>(((b + 255) / 256) * 256); }
+
+size_t gemm_ws_bytes(int64_t M, int64_t N) {
+    if (M <= kDecodeMaxM) return round256(decode::workspace_bytes(N / 128));
+    return 0;
+}
+
+size_t act_ws_bytes(int64_t M, int64_t K) { return round256(M * K) + round256(M * (K / 128) * 4); }
+
+// ---------------------------------------------------------------- launches
+
+cudaError_t launch_quantize_act(const DeviceInfo &d, const void *x, int64_t M, int64_t K,
+                                uint8_t *q, float *sa, cudaStream_t st) {
+    const int64_t groups = M * (K / 128);
+    const int64_t teams_needed = (groups + kActUnroll - 1) / kActUnroll;
+    const int64_t blocks_needed = (teams_needed * 16 + kActThreads - 1) / kActThreads;
+    const int64_t max_blocks = static_cast<int64_t>(d.sm_count) * (2048 / kActThreads);
+    const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
+    quantize_act_kernel<<<blocks, kActThreads, 0, st>>>(static_cast<const uint4 *>(x), groups,
+                                                       reinterpret_cast<uint2 *>(q), sa);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
+                        const uint8_t *qw, const float *sw, int64_t M, int64_t N, int64_t K,
+                        void *y, void *ws, cudaStream_t st, fp8bq_status *err) {
+    *err = FP8BQ_OK;
+    if (M <= kDecodeMaxM) {
+        CUtensorMap tw, tx;
+        if (!make_tmap(&tw, qw, N, K, decode::BNW) || !make_tmap(&tx, qa, M, K, decode::MT)) {
+            *err = FP8BQ_ERR_CUDA;
+            return cudaSuccess;
+        }
+        const int64_t NB = N / 128;
+        const int64_t units = NB * (K / 128);
+        int64_t grid = d.sm_count;
+        if (grid > decode::kMaxGrid) grid = decode::kMaxGrid;
+        if (grid > units) grid = units;
+        int *counters = static_cast<int *>(ws);
+        float *partials =
+            reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::counters_bytes(NB));
+        decode::gemm_decode_kernel<<<static_cast<int>(grid), decode::kNumThreads,
+                                     decode::Layout::kDynamicSmem, st>>>(
+            tw, tx, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
+            static_cast<int>(N), static_cast<int>(K), counters, partials, d.status);
+    } else {
+        CUtensorMap ta, tb;
+        if (!make_tmap(&ta, qa, M, K, prefill::BM) || !make_tmap(&tb, qw, N, K, kPrefillBN)) {
+            *err = FP8BQ_ERR_CUDA;
+            return cudaSuccess;
+        }
+        const int64_t tiles = ((M + prefill::BM - 1) / prefill::BM) * ((N + kPrefillBN - 1) / kPrefillBN);
+        const int grid = static_cast<int>(tiles < d.sm_count ? tiles : d.sm_count);
+        prefill::gemm_prefill_kernel<kPrefillBN>
+            <<<grid, prefill::kNumThreads, prefill::Layout<kPrefillBN>::kDynamicSmem, st>>>(
+                ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
+                static_cast<int>(N), static_cast<int>(K), d.status);
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace fp8bq
+
+using namespace fp8bq;
+
+extern "C" {
+
+fp8bq_status fp8bq_quantize_act(const void *x_bf16, int64_t M, int64_t K, uint8_t *q_e4m3,
+                                float *sa, void *stream) {
+    fp8bq_status st = check_mk(M, K);
+    if (st != FP8BQ_OK) return st;
+    if (M == 0) return FP8BQ_OK;
+    if (!x_bf16 || !q_e4m3 || !sa) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(q_e4m3) || !aligned16(sa)) return FP8BQ_ERR_MISALIGNED;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    return from_cuda(launch_quantize_act(*d, x_bf16, M, K, q_e4m3, sa,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+fp8bq_status fp8bq_quantize_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *q_e4m3,
+                                   float *sw, void *stream) {
+    fp8bq_status st = check_mk(N, K);
+    if (st != FP8BQ_OK) return st;
+    if (N <= 0 || N % 128 != 0) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    if (N / 128 > 65535) return FP8BQ_ERR_UNSUPPORTED_SHAPE;  // grid.y limit
+    if (!w_bf16 || !q_e4m3 || !sw) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(w_bf16) || !aligned16(q_e4m3) || !aligned16(sw)) return FP8BQ_ERR_MISALIGNED;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    const dim3 grid(static_cast<unsigned>(K / 128), static_cast<unsigned>(N / 128));
+    quantize_weight_kernel<<<grid, kWeightThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t *>(w_bf16), K, q_e4m3, sw);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return from_cuda(cudaGetLastError());
+}
+
+size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {
+    if (check_mnk(M, N, K) != FP8BQ_OK || M == 0) return 0;
+    if (op == FP8BQ_OP_GEMM) return gemm_ws_bytes(M, N);
+    if (op == FP8BQ_OP_LINEAR) return act_ws_bytes(M, K) + gemm_ws_bytes(M, N);
+    return 0;
+}
+
+fp8bq_status fp8bq_gemm(const uint8_t *qa, const float *sa, const uint8_t *qw, const float *sw,
+                        int64_t M, int64_t N, int64_t K, void *y_bf16, void *workspace,
+                        size_t ws_bytes, void *stream) {
+    fp8bq_status st = check_mnk(M, N, K);
+    if (st != FP8BQ_OK) return st;
+    if (M == 0) return FP8BQ_OK;
+    if (!qa || !sa || !qw || !sw || !y_bf16) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16))
+        return FP8BQ_ERR_MISALIGNED;
+    const size_t need = gemm_ws_bytes(M, N);
+    if (need && (!workspace || ws_bytes < need)) return FP8BQ_ERR_WORKSPACE;
+    if (need && !aligned16(workspace)) return FP8BQ_ERR_MISALIGNED;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    fp8bq_status err;
+    cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, workspace,
+                                static_cast<cudaStream_t>(stream), &err);
+    if (err != FP8BQ_OK) return err;
+    return from_cuda(e);
+}
+
+fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const float *sw, int64_t M,
+                          int64_t N, int64_t K, void *y_bf16, void *workspace, size_t ws_bytes,
+                          void *stream) {
+    fp8bq_status st = check_mnk(M, N, K);
+    if (st != FP8BQ_OK) return st;
+    if (M == 0) return FP8BQ_OK;
+    if (!x_bf16 || !qw || !sw || !y_bf16) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16))
+        return FP8BQ_ERR_MISALIGNED;
+    const size_t need = act_ws_bytes(M, K) + gemm_ws_bytes(M, N);
+    if (!workspace || ws_bytes < need) return FP8BQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP8BQ_ERR_MISALIGNED;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint8_t *qa = ws;
+    float *sa = reinterpret_cast<float *>(ws + round256(M * K));
+    void *gemm_ws = ws + act_ws_bytes(M, K);
+    cudaError_t e = launch_quantize_act(*d, x_bf16, M, K, qa, sa, s);
+    if (e != cudaSuccess) return FP8BQ_ERR_CUDA;
+    fp8bq_status err;
+    e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, gemm_ws, s, &err);
+    if (err != FP8BQ_OK) return err;
+    return from_cuda(e);
+}
+
+fp8bq_status fp8bq_workspace_init(void *workspace, size_t ws_bytes, void *stream) {
+    if (ws_bytes == 0) return FP8BQ_OK;
+    if (!workspace) return FP8BQ_ERR_INVALID_ARG;
+    return from_cuda(cudaMemsetAsync(workspace, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+fp8bq_status fp8bq_last_device_status(void *stream) {
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FP8BQ_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, d->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FP8BQ_ERR_CUDA;
+    if (v != 0 && cudaMemset(d->status, 0, sizeof(int)) != cudaSuccess) return FP8BQ_ERR_CUDA;
+    return v == 0 ? FP8BQ_OK : static_cast<fp8bq_status>(v);
+}
+
+const char *fp8bq_status_string(fp8bq_status status) {
+    switch (status) {
+        case FP8BQ_OK: return "ok";
+        case FP8BQ_ERR_INVALID_ARG: return "invalid argument (null pointer or negative size)";
+        case FP8BQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (N and K must be multiples of 128)";
+        case FP8BQ_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case FP8BQ_ERR_WORKSPACE: return "workspace missing or too small";
+        case FP8BQ_ERR_CUDA: return "CUDA runtime or driver call failed";
+        case FP8BQ_ERR_TIMEOUT: return "a kernel abandoned a bounded wait (timeout)";
+        case FP8BQ_ERR_NO_DEVICE: return "no sm_100 device is current";
+    }
+    return "unknown status";
+}
+
+uint64_t fp8bq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int fp8bq_version(void) { return 100; }
+
+}  // extern "C"

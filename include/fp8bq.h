@@ -1,0 +1,162 @@
+/*
+ * fp8bq.h -- C ABI of the B200 (sm_100a) W8A8 FP8 block-scaled linear layer.
+ *
+ * The method (page "ProCreations/Nanbeige4.3-33B-FP8", introduction and section
+ * "Recipe and calibration"): linear layers run in W8A8 FP8 -- E4M3 weights with
+ * one scale per 128x128 block (standard min-max, data independent) and
+ * activations quantized dynamically per token and per group of 128 channels;
+ * embeddings and the output head stay BF16 and are not part of this library.
+ *
+ * Numerics fixed by this library (the page leaves them open):
+ *   - E4M3 is the OCP "e4m3fn" format (largest finite value 448, no infinities).
+ *   - scale = amax / 448 computed as one IEEE binary32 division (round to
+ *     nearest even); a group or block whose amax is 0 gets scale 1.0.
+ *   - code = E4M3 round-to-nearest-even of fl32(x / scale), saturating at
+ *     +-448; the sign of zero is kept; finite input never yields the NaN code.
+ *   - the GEMM multiplies E4M3 codes exactly, sums each 128-wide K chunk in
+ *     FP32, promotes the chunk into an FP32 accumulator multiplied by
+ *     act_scale[m, kb] * weight_scale[n/128, kb], and rounds the result to BF16
+ *     (round to nearest even).  Y = X W^T (W stored out x in, nn.Linear layout).
+ *
+ * Layouts: every matrix is dense and row-major (leading dimension = number of
+ * columns).  X, Y: BF16 [M, K] / [M, N].  Codes: one byte per element, E4M3
+ * bit patterns.  Activation scales: FP32 [M, K/128].  Weight scales: FP32
+ * [N/128, K/128].
+ *
+ * Ownership: the caller allocates and frees every buffer (inputs, outputs and
+ * workspace) in device memory of the current device; the library never
+ * allocates device memory and keeps no per-buffer state on the host (TMA
+ * descriptors are encoded on every call and passed by value to the kernels).
+ *
+ * Execution: every compute call is asynchronous on the given stream (a
+ * cudaStream_t passed as void*; NULL = the legacy default stream) and returns
+ * after enqueueing.  Argument errors are detected on the host before anything
+ * is enqueued and reported synchronously.  A kernel that gives up on an
+ * internal wait (FP8BQ_ERR_TIMEOUT) records it in a per-device status word,
+ * read by fp8bq_last_device_status().
+ *
+ * Requirements checked on the host (else the listed status, nothing enqueued):
+ *   M >= 0, N > 0, K > 0, N % 128 == 0, K % 128 == 0  (else UNSUPPORTED_SHAPE;
+ *     M == 0 is a no-op returning FP8BQ_OK);
+ *   M, N, K <= 2^31 - 1 and every tensor smaller than 2^40 bytes (UNSUPPORTED_SHAPE);
+ *   non-NULL pointers for every non-empty tensor (INVALID_ARG);
+ *   every pointer 16-byte aligned (MISALIGNED);
+ *   workspace at least fp8bq_workspace_size(...) bytes (WORKSPACE).
+ * Inputs must be finite; NaN or infinite inputs give unspecified codes.
+ *
+ * Thread safety: calls on different streams may run concurrently as long as
+ * they use different output and workspace buffers.
+ */
+#ifndef FP8BQ_H
+#define FP8BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Symbols of this ABI are the only ones the shared library exports. */
+#if defined(__GNUC__)
+#define FP8BQ_API __attribute__((visibility("default")))
+#else
+#define FP8BQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8BQ_OK = 0,
+    FP8BQ_ERR_INVALID_ARG = 1,       /* NULL pointer or negative size */
+    FP8BQ_ERR_UNSUPPORTED_SHAPE = 2, /* N or K not a multiple of 128, or too large */
+    FP8BQ_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+    FP8BQ_ERR_WORKSPACE = 4,         /* workspace missing or smaller than required */
+    FP8BQ_ERR_CUDA = 5,              /* a CUDA runtime or driver call failed */
+    FP8BQ_ERR_TIMEOUT = 6,           /* a kernel abandoned a bounded wait */
+    FP8BQ_ERR_NO_DEVICE = 7          /* no sm_100 device is current */
+} fp8bq_status;
+
+/* Operation selector for fp8bq_workspace_size. */
+typedef enum { FP8BQ_OP_GEMM = 0, FP8BQ_OP_LINEAR = 1 } fp8bq_op;
+
+/*
+ * Dynamic per-token, group-128 activation quantization (page
+ * "ProCreations/Nanbeige4.3-33B-FP8", introduction: activations get one scale
+ * per token and per 128-channel group, computed at run time).
+ *   x_bf16 : in,  BF16 [M, K]
+ *   q_e4m3 : out, E4M3 codes [M, K]
+ *   sa     : out, FP32 [M, K/128]; sa[m, g] = amax(|x[m, 128g : 128g+128]|) / 448, or 1
+ * Codes and scales are bit-exact with the definition above.
+ */
+FP8BQ_API fp8bq_status fp8bq_quantize_act(const void *x_bf16, int64_t M, int64_t K, uint8_t *q_e4m3,
+                                float *sa, void *stream);
+
+/*
+ * Offline 128x128-block min-max weight quantization (same page, section
+ * "Recipe and calibration": one scale per 128x128 block of the E4M3 weights,
+ * chosen by plain min-max without calibration data).
+ *   w_bf16 : in,  BF16 [N, K] (out x in)
+ *   q_e4m3 : out, E4M3 codes [N, K]
+ *   sw     : out, FP32 [N/128, K/128]; sw[i, j] = amax of block (i, j) / 448, or 1
+ * Codes and scales are bit-exact with the definition above.
+ */
+FP8BQ_API fp8bq_status fp8bq_quantize_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *q_e4m3,
+                                   float *sw, void *stream);
+
+/*
+ * Block-scaled FP8 GEMM (same page, introduction: W8A8 FP8 linear layers with
+ * BF16 activations in and out): Y[m, n] = BF16( sum_kb sa[m,kb] sw[n/128,kb]
+ * sum_{k in kb} e4m3(qa[m,k]) e4m3(qw[n,k]) ).
+ *   qa, sa : in, activation codes [M, K] and scales [M, K/128]
+ *   qw, sw : in, weight codes [N, K] and scales [N/128, K/128]
+ *   y_bf16 : out, BF16 [M, N]
+ *   workspace, ws_bytes : device scratch of at least
+ *       fp8bq_workspace_size(FP8BQ_OP_GEMM, M, N, K) bytes (may be NULL when
+ *       that is 0).  Its first fp8bq_workspace_size(...) bytes must hold the
+ *       state left by fp8bq_workspace_init() or by a previous successful call;
+ *       calls that share a workspace must be ordered (same stream).
+ * Output accuracy: |y - ref| <= 1e-2 |ref| + 2e-3 rms(ref) against the FP64 sum
+ * of the dequantized operands; results are deterministic for a given shape.
+ */
+FP8BQ_API fp8bq_status fp8bq_gemm(const uint8_t *qa, const float *sa, const uint8_t *qw, const float *sw,
+                        int64_t M, int64_t N, int64_t K, void *y_bf16, void *workspace,
+                        size_t ws_bytes, void *stream);
+
+/*
+ * Linear layer with the activation quantization fused into the call:
+ * Y = gemm(quantize_act(X), qw, sw) with identical codes and scales.
+ *   x_bf16 : in, BF16 [M, K]; qw / sw / y_bf16 as in fp8bq_gemm
+ *   workspace : at least fp8bq_workspace_size(FP8BQ_OP_LINEAR, M, N, K) bytes,
+ *               same state rule as fp8bq_gemm.
+ */
+FP8BQ_API fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const float *sw, int64_t M,
+                          int64_t N, int64_t K, void *y_bf16, void *workspace, size_t ws_bytes,
+                          void *stream);
+
+/* Bytes of workspace the operation needs for this shape (0 when none, and for
+ * arguments the call would reject).  Always a multiple of 256. */
+FP8BQ_API size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K);
+
+/* Put a workspace into its initial state (zero-fills ws_bytes bytes on the
+ * stream).  Needed once after allocation and after a call that reported
+ * FP8BQ_ERR_TIMEOUT. */
+FP8BQ_API fp8bq_status fp8bq_workspace_init(void *workspace, size_t ws_bytes, void *stream);
+
+/* Synchronizes the stream, then returns and clears the current device's status
+ * word: FP8BQ_OK, or FP8BQ_ERR_TIMEOUT if a kernel abandoned a wait since the
+ * last read.  A failed synchronize returns FP8BQ_ERR_CUDA. */
+FP8BQ_API fp8bq_status fp8bq_last_device_status(void *stream);
+
+/* Static description of a status code (never NULL). */
+FP8BQ_API const char *fp8bq_status_string(fp8bq_status status);
+
+/* Number of kernels this library has launched in this process (all devices). */
+FP8BQ_API uint64_t fp8bq_launch_count(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+FP8BQ_API int fp8bq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BQ_H */

@@ -1,0 +1,154 @@
+"""Host-side checks of the C ABI (no kernel is launched).
+
+* the library builds and loads, and exports every function include/fp8bq.h declares;
+* argument errors are reported synchronously with the documented status codes
+  (shape, NULL, alignment, workspace), before any device work;
+* workspace sizes and status strings are well defined.
+On a machine without a GPU, a call with valid arguments reports
+FP8BQ_ERR_NO_DEVICE; that check is skipped when a GPU is present (the
+pointers used here are fake).
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import fp8_block_scaled_09_b200 as fp8bq
+from fp8_block_scaled_09_b200 import build as fp8bq_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "fp8bq.h")
+
+OK, INVALID, SHAPE, MISALIGNED, WORKSPACE, CUDA, TIMEOUT, NODEV = range(8)
+
+
+@pytest.fixture(scope="module")
+def L():
+    fp8bq_build.build()
+    return fp8bq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8bq_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
+              "fp8bq_workspace_size", "fp8bq_last_device_status", "fp8bq_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", fp8bq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (fp8bq_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert getattr(L, n) is not None
+
+
+def test_only_the_abi_is_exported(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", fp8bq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    ours = set(re.findall(r"\bT (\w+)", out))
+    extra = sorted(n for n in ours if not n.startswith("fp8bq_"))
+    # cudart (linked statically) keeps its symbols hidden; nothing else leaks
+    assert not [n for n in extra if "fp8bq" in n.lower()], extra
+
+
+def test_status_strings(L):
+    for code in range(8):
+        assert len(fp8bq.status_string(code)) > 0
+    assert fp8bq.status_string(99) == "unknown status"
+    assert L.fp8bq_version() == 100
+
+
+P = ctypes.c_void_p
+GOOD = P(0x10000)       # fake, 16-byte aligned
+ODD = P(0x10008)        # fake, misaligned
+
+
+def test_quantize_act_argument_errors(L):
+    f = L.fp8bq_quantize_act
+    assert f(GOOD, 4, 100, GOOD, GOOD, None) == SHAPE       # K % 128
+    assert f(GOOD, -1, 128, GOOD, GOOD, None) == SHAPE
+    assert f(GOOD, 4, 0, GOOD, GOOD, None) == SHAPE
+    assert f(GOOD, 4, 1 << 40, GOOD, GOOD, None) == SHAPE  # too large
+    assert f(None, 0, 128, None, None, None) == OK           # M == 0 is a no-op
+    assert f(None, 4, 128, GOOD, GOOD, None) == INVALID
+    assert f(GOOD, 4, 128, None, GOOD, None) == INVALID
+    assert f(GOOD, 4, 128, GOOD, None, None) == INVALID
+    assert f(ODD, 4, 128, GOOD, GOOD, None) == MISALIGNED
+    assert f(GOOD, 4, 128, ODD, GOOD, None) == MISALIGNED
+    assert f(GOOD, 4, 128, GOOD, ODD, None) == MISALIGNED
+
+
+def test_quantize_weight_argument_errors(L):
+    f = L.fp8bq_quantize_weight
+    assert f(GOOD, 100, 128, GOOD, GOOD, None) == SHAPE     # N % 128
+    assert f(GOOD, 0, 128, GOOD, GOOD, None) == SHAPE
+    assert f(GOOD, 128, 200, GOOD, GOOD, None) == SHAPE
+    assert f(None, 128, 128, GOOD, GOOD, None) == INVALID
+    assert f(GOOD, 128, 128, ODD, GOOD, None) == MISALIGNED
+
+
+def test_gemm_argument_errors(L):
+    f = L.fp8bq_gemm
+    ws = fp8bq.workspace_size(fp8bq.OP_GEMM, 8, 256, 256)
+    assert f(GOOD, GOOD, GOOD, GOOD, 8, 200, 256, GOOD, GOOD, ws, None) == SHAPE
+    assert f(GOOD, GOOD, GOOD, GOOD, 8, 256, 250, GOOD, GOOD, ws, None) == SHAPE
+    assert f(GOOD, GOOD, GOOD, GOOD, 8, 0, 256, GOOD, GOOD, ws, None) == SHAPE
+    assert f(None, None, None, None, 0, 256, 256, None, None, 0, None) == OK
+    assert f(GOOD, None, GOOD, GOOD, 8, 256, 256, GOOD, GOOD, ws, None) == INVALID
+    assert f(GOOD, GOOD, GOOD, GOOD, 8, 256, 256, None, GOOD, ws, None) == INVALID
+    assert f(GOOD, GOOD, ODD, GOOD, 8, 256, 256, GOOD, GOOD, ws, None) == MISALIGNED
+    assert f(GOOD, GOOD, GOOD, GOOD, 8, 256, 256, GOOD, None, ws, None) == WORKSPACE
+    assert f(GOOD, GOOD, GOOD, GOOD, 8, 256, 256, GOOD, GOOD, ws - 1, None) == WORKSPACE
+    assert f(GOOD, GOOD, GOOD, GOOD, 8, 256, 256, GOOD, ODD, ws, None) == MISALIGNED
+
+
+def test_linear_argument_errors(L):
+    f = L.fp8bq_linear
+    ws = fp8bq.workspace_size(fp8bq.OP_LINEAR, 300, 256, 256)
+    assert f(GOOD, GOOD, GOOD, 300, 256, 100, GOOD, GOOD, ws, None) == SHAPE
+    assert f(GOOD, GOOD, None, 300, 256, 256, GOOD, GOOD, ws, None) == INVALID
+    assert f(ODD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws, None) == MISALIGNED
+    assert f(GOOD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws - 256, None) == WORKSPACE
+    assert f(None, None, None, 0, 256, 256, None, None, 0, None) == OK
+
+
+def test_workspace_sizes(L):
+    g = lambda M, N, K: fp8bq.workspace_size(fp8bq.OP_GEMM, M, N, K)
+    lin = lambda M, N, K: fp8bq.workspace_size(fp8bq.OP_LINEAR, M, N, K)
+    assert g(0, 256, 256) == 0 and lin(0, 256, 256) == 0
+    assert g(8, 200, 256) == 0 and g(8, 256, 200) == 0           # rejected shapes
+    assert fp8bq.workspace_size(7, 8, 256, 256) == 0              # unknown op
+    assert g(8192, 9216, 7168) == 0                              # prefill GEMM needs none
+    d = g(16, 9216, 7168)
+    assert d > 0 and d % 256 == 0
+    # decode split-K: counters + (N/128 + 256) slots of 16 x 128 FP32 partials
+    assert d >= (72 + 256) * 16 * 128 * 4
+    # linear adds the activation codes and scales
+    assert lin(8192, 9216, 7168) >= 8192 * 7168 + 8192 * 56 * 4
+    assert lin(16, 9216, 7168) >= d + 16 * 7168 + 16 * 56 * 4
+    for args in ((1, 128, 128), (17, 384, 1024), (4096, 7168, 21504)):
+        assert lin(*args) % 256 == 0 and g(*args) % 256 == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="valid calls would launch kernels on fake pointers")
+def test_valid_call_without_device_reports_no_device(L):
+    assert L.fp8bq_quantize_act(GOOD, 4, 128, GOOD, GOOD, None) == NODEV
+    assert L.fp8bq_last_device_status(None) == NODEV
+
+
+def test_binding_fails_loudly_without_cuda_tensors():
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fp8bq.quantize_act(x)

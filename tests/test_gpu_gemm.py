@@ -1,0 +1,180 @@
+"""GPU parity of the block-scaled GEMM and the fused linear layer.
+
+The GEMM is fed the oracle's codes and scales; its BF16 output must satisfy
+|y - ref| <= 1e-2 |ref| + 2e-3 rms(ref) against the oracle's FP64 sum of the
+dequantized operands (tolerance of the library's accuracy contract; the page
+"ProCreations/Nanbeige4.3-33B-FP8", "Compatibility and limitations", claims no
+bit-exact equivalence across kernel geometry).  Shapes span several tiles with
+ragged M tails on both the decode (M <= 16) and prefill paths; the full
+workload shapes are checked on sampled rows.  In the exact-arithmetic regime
+(small-integer codes, power-of-two scales) every partial sum is exact in FP32,
+so the output must equal the BF16 rounding of the exact result bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fp8_block_scaled_09_b200 as fp8bq
+import oracle
+import workloads
+from gpu_util import Guarded, bf16_to_f64, to_dev_codes, to_dev_f32, tolerance_report
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    fp8bq.lib()
+    yield
+    assert fp8bq.last_device_status() == 0
+
+
+def operands(M, N, K, seed, x=None):
+    if x is None:
+        x = workloads.activation(M, K, seed, outliers=max(1, K // 1024))
+    w = workloads.weight(N, K, seed + 1)
+    qa, sa = oracle.quantize_act(x)
+    qw, sw = oracle.quantize_weight(w)
+    return x, qa, sa, qw, sw
+
+
+def run_gemm(qa, sa, qw, sw):
+    M, K = qa.shape
+    N = qw.shape[0]
+    y = Guarded((M, N), torch.bfloat16)
+    ws = fp8bq.new_workspace(fp8bq.OP_GEMM, M, N, K, "cuda")
+    fp8bq.gemm(to_dev_codes(qa), to_dev_f32(sa), to_dev_codes(qw), to_dev_f32(sw), out=y.t,
+               workspace=ws)
+    torch.cuda.synchronize()
+    assert y.guards_intact()
+    return y.t
+
+
+def check(y, ref):
+    ok, ratio, rms = tolerance_report(y, ref)
+    assert ok, f"worst error / bound = {ratio:.3f} (rms(ref) = {rms:.4g})"
+
+
+DECODE_SHAPES = [(1, 128, 128), (1, 1024, 7168), (2, 256, 384), (4, 9216, 7168),
+                 (8, 7168, 7168), (15, 384, 1024), (16, 1024, 7168), (16, 128, 21504),
+                 (3, 16384, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
+def test_gemm_decode_path(M, N, K):
+    _, qa, sa, qw, sw = operands(M, N, K, 100 + M)
+    y = run_gemm(qa, sa, qw, sw)
+    check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
+
+
+PREFILL_SHAPES = [(17, 128, 128), (128, 256, 256), (129, 384, 1024), (255, 1152, 512),
+                  (1000, 512, 896), (300, 128, 7168), (2048, 2048, 384)]
+
+
+@pytest.mark.parametrize("M,N,K", PREFILL_SHAPES)
+def test_gemm_prefill_path(M, N, K):
+    _, qa, sa, qw, sw = operands(M, N, K, 200 + M)
+    y = run_gemm(qa, sa, qw, sw)
+    check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
+
+
+def sample_rows(M, step, extra=()):
+    rows = set(range(0, M, step)) | {M - 1} | set(r for r in extra if 0 <= r < M)
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+@pytest.mark.parametrize("name", ["k_proj", "qkv_m8", "o_proj_m4", "qkv_prefill", "fc",
+                                  "gate_up", "down", "o_proj_long"])
+def test_gemm_full_workloads_sampled(name):
+    g = workloads.by_name(name)
+    x = g.make_x()
+    qa, sa = oracle.quantize_act(x)
+    qw, sw = oracle.quantize_weight(g.make_w())
+    y = run_gemm(qa, sa, qw, sw)
+    step = 1 if g.M <= 16 else max(1, g.M // 48)
+    rows = sample_rows(g.M, step, extra=(127, 128, g.M - 129))
+    ref = oracle.gemm_ref(qa, sa, qw, sw, rows=rows)
+    check(bf16_to_f64(y)[rows], ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(4, 256, 512), (300, 384, 640)])
+def test_gemm_exact_arithmetic_regime_bit_exact(M, N, K):
+    rng = np.random.default_rng(M)
+    small = np.array([0x00, 0x38, 0x40, 0x44, 0x48, 0xB8, 0xC0, 0xC4], np.uint8)  # 0,+-1,+-2,+-3,4
+    qa = rng.choice(small, size=(M, K))
+    qw = rng.choice(small, size=(N, K))
+    sa = np.ldexp(np.float32(1.0), rng.integers(-3, 3, size=(M, K // 128))).astype(np.float32)
+    sw = np.ldexp(np.float32(1.0), rng.integers(-3, 3, size=(N // 128, K // 128))).astype(np.float32)
+    y = run_gemm(qa, sa, qw, sw)
+    ref = oracle.gemm_ref(qa, sa, qw, sw)            # exact: |sums| < 2^24 at these sizes
+    expect = oracle.bf16_round(ref)
+    got = y.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, expect)
+
+
+def test_gemm_identity_weight_closed_form():
+    M = 200
+    x = workloads.activation(M, 128, 21, outliers=1)
+    qa, sa = oracle.quantize_act(x)
+    qw, sw = oracle.quantize_weight(torch.eye(128, dtype=torch.bfloat16))
+    y = run_gemm(qa, sa, qw, sw)
+    # Y[m, n] = BF16(dq(qa[m, n]) * fl32(sa[m] * sw)) * 448 ... evaluated by the oracle in FP64
+    check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
+
+
+@pytest.mark.parametrize("M", [8, 600])
+def test_gemm_deterministic(M):
+    _, qa, sa, qw, sw = operands(M, 1024, 7168, 7)
+    y1 = run_gemm(qa, sa, qw, sw).cpu()
+    y2 = run_gemm(qa, sa, qw, sw).cpu()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_gemm_empty_m_is_noop():
+    qa = torch.zeros((0, 256), dtype=torch.uint8, device="cuda")
+    sa = torch.zeros((0, 2), dtype=torch.float32, device="cuda")
+    qw = torch.zeros((128, 256), dtype=torch.uint8, device="cuda")
+    sw = torch.ones((1, 2), dtype=torch.float32, device="cuda")
+    y = fp8bq.gemm(qa, sa, qw, sw)
+    assert y.shape == (0, 128)
+
+
+# ------------------------------------------------------------------ fused linear
+
+@pytest.mark.parametrize("M,N,K", [(1, 1024, 7168), (16, 1024, 7168), (5, 384, 640),
+                                   (33, 256, 1024), (700, 384, 7168)])
+def test_linear_matches_oracle_and_unfused_path(M, N, K):
+    x, qa, sa, qw, sw = operands(M, N, K, 300 + M)
+    xd = x.cuda()
+    y = Guarded((M, N), torch.bfloat16)
+    ws = fp8bq.new_workspace(fp8bq.OP_LINEAR, M, N, K, "cuda")
+    fp8bq.linear(xd, to_dev_codes(qw), to_dev_f32(sw), out=y.t, workspace=ws)
+    torch.cuda.synchronize()
+    assert y.guards_intact()
+    check(bf16_to_f64(y.t), oracle.linear_ref(x, qw, sw))
+    # same codes and scales as the standalone quantizer feeding the standalone GEMM
+    gq, gs = fp8bq.quantize_act(xd)
+    y2 = fp8bq.gemm(gq, gs, to_dev_codes(qw), to_dev_f32(sw))
+    assert torch.equal(y.t.view(torch.int16), y2.view(torch.int16))
+
+
+def test_linear_kproj_workload_with_zero_row():
+    g = workloads.KPROJ_M16
+    x = g.make_x()
+    qw, sw = oracle.quantize_weight(g.make_w())
+    y = fp8bq.linear(x.cuda(), to_dev_codes(qw), to_dev_f32(sw))
+    torch.cuda.synchronize()
+    yf = bf16_to_f64(y)
+    check(yf, oracle.linear_ref(x, qw, sw))
+    assert np.all(yf[g.M - 1] == 0.0)          # the all-zero activation row
+
+
+def test_linear_prefill_qkv_sampled():
+    g = workloads.PREFILL_QKV
+    x = g.make_x()
+    qw, sw = oracle.quantize_weight(g.make_w())
+    y = fp8bq.linear(x.cuda(), to_dev_codes(qw), to_dev_f32(sw))
+    torch.cuda.synchronize()
+    rows = sample_rows(g.M, 256, extra=(128, 4095, 4096))
+    check(bf16_to_f64(y)[rows], oracle.linear_ref(x, qw, sw, rows=rows))
