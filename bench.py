@@ -1,0 +1,563 @@
+#!/usr/bin/env python
+"""Throughput of the W8A8 FP8 block-scaled linear layer on B200.
+
+One JSON line on rank 0.  A *step* is one pass of the hot path over the decode
+GEMV set: fp8bq_linear (dynamic group-128 activation quantization fused into
+the call, block-scaled FP8 GEMM, BF16 out) for M in {1, 4, 8} tokens against
+the fused QKV weight [9216, 7168] and the o_proj weight [7168, 7168] -- six
+linear layers per step.  The weights are quantized once (the offline half of
+the method) and rotated over four device copies per shape so that every step
+streams them from HBM (4 x 66 MB and 4 x 51 MB, larger than the 126 MB L2).
+
+``value`` is algorithmic HBM bytes per second (weight codes + weight scales +
+BF16 activations + BF16 outputs; one pass over each), timed with CUDA events
+around CUDA-graph replays of the steps, max over ranks.  Alongside:
+
+* ``roofline``   the decode GEMM kernel alone (pre-quantized activations),
+                 algorithmic bytes / its average launch time vs measured HBM.
+* ``prefill``    fp8bq_linear and the GEMM kernel on the prefill fused-QKV
+                 shape X[8192, 7168] W[9216, 7168], TFLOP/s (2 M N K) vs the
+                 measured dense-FP8 peak (measured BF16 x 2), L2 flushed
+                 between iterations.
+* ``quantize_act`` on [32768, 7168] (long-prefill activation), GB/s.
+* ``workloads``  GEMM-kernel and linear throughput for every other shape.
+* ``e2e``        the same decode steps through the public API from pinned host
+                 buffers: H2D copy of X, the linear call, D2H copy of Y.
+* ``cpu_baseline`` the CPU oracle (plain C, FP64 GEMM) on full decode steps.
+
+``--impl reference`` times the CPU oracle instead, on the same metric.
+``--gpus N`` (under torchrun) runs N independent replicas, one per GPU: the
+layer has no exchange step, so there is no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "FP8 block-scaled GEMM TFLOPS (prefill) & HBM GB/s (decode), % of roofline, 1 B200"
+FP8_OVER_BF16 = 2.0          # nominal dense ratio 4.5 / 2.25 PFLOP/s
+ROTATE = 4                   # device copies of each decode weight
+DECODE_WORKLOAD = ("decode GEMV set: fp8bq_linear, M in {1,4,8} x {fused QKV W[9216,7168], "
+                   "o_proj W[7168,7168]}, E4M3 128x128-blocked weights, X BF16 N(0,1) with "
+                   "7 outlier channels x20")
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def linear_bytes(g: W.Gemm) -> int:
+    """Algorithmic bytes of one linear: W codes, W scales, BF16 X in, BF16 Y out."""
+    return g.N * g.K + (g.N // 128) * (g.K // 128) * 4 + g.M * g.K * 2 + g.M * g.N * 2
+
+
+def gemm_bytes(g: W.Gemm) -> int:
+    """Algorithmic bytes of one GEMM launch: W and X codes, both scale sets, BF16 Y."""
+    return (g.N * g.K + (g.N // 128) * (g.K // 128) * 4 + g.M * g.K + g.M * (g.K // 128) * 4
+            + g.M * g.N * 2)
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML on a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device_index: int):
+        self.samples: list[tuple[int, int]] = []
+        self.max_mhz = None
+        self._on = False
+        self._thread = None
+        self.error = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 -- clocks are reported as unavailable
+            self.error = f"{type(e).__name__}: {e}"
+            self._h = None
+
+    def _run(self):
+        nv = self._nvml
+        while self._on:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((mhz, rs))
+            except Exception as e:  # noqa: BLE001
+                self.error = str(e)
+                return
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._on = True
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._on = False
+        if self._thread is not None:
+            self._thread.join()
+            # one sample right after the region, so short regions still get one
+            try:
+                self.samples.append((self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM),
+                                     self._nvml.nvmlDeviceGetCurrentClocksEventReasons(self._h)))
+            except Exception:  # noqa: BLE001
+                pass
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml", "error": self.error}
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = sorted(n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml, 2 ms polling during the timed regions"}
+
+
+def events_ms(torch, fn, iters: int) -> float:
+    s = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for i in range(iters):
+        fn(i)
+    e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def flushed_ms(torch, fn, iters: int, warmup: int, flush) -> list[float]:
+    """Per-iteration event times with an L2 flush (untimed) before each iteration."""
+    s = torch.cuda.current_stream()
+    evs = []
+    for i in range(warmup + iters):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        fn()
+        e1.record(s)
+        if i >= warmup:
+            evs.append((e0, e1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def decode_host_inputs():
+    """Host BF16 activations and weights of the decode set (seeded)."""
+    xs = [g.make_x() for g in W.DECODE_SET]
+    ws = {}
+    for g in W.DECODE_SET:
+        if g.N not in ws:
+            ws[g.N] = g.make_w()
+    return xs, ws
+
+
+def oracle_decode_steps(oracle, xs, qws, steps: int, col_frac: float = 1.0):
+    """Runs `steps` decode steps of the oracle; returns (seconds, algorithmic bytes)."""
+    total_bytes = 0
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        for g, x in zip(W.DECODE_SET, xs):
+            qw, sw = qws[g.N]
+            nb = max(1, int(round(col_frac * (g.N // 128))))
+            n = nb * 128
+            oracle.linear_ref(x, qw[:n], sw[:nb])
+            total_bytes += linear_bytes(W.scaled(g, N=n)) if n != g.N else linear_bytes(g)
+    return time.perf_counter() - t0, total_bytes
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    xs, ws = decode_host_inputs()
+    qws = {N: oracle.quantize_weight(w) for N, w in ws.items()}    # offline step, untimed
+    # size each step so the whole run stays within about two minutes
+    t_one, _ = oracle_decode_steps(oracle, xs, qws, 1)
+    budget_s = 120.0
+    frac = min(1.0, budget_s / max(1e-9, (args.steps + args.warmup) * t_one))
+    oracle_decode_steps(oracle, xs, qws, args.warmup, frac)
+    secs, nbytes = oracle_decode_steps(oracle, xs, qws, args.steps, frac)
+    gbs = nbytes / secs / 1e9
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"each step: the 6 decode linears on {frac:.3f} of the output columns "
+              "(whole n-blocks), all rows and all K; oracle.linear_ref (plain C, OpenMP, "
+              "binary32 quantizer + FP64 GEMM)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded numpy PCG64, BF16)",
+        "config": {"workload": DECODE_WORKLOAD, "device": "host CPU"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import fp8_block_scaled_09_b200 as fp8bq
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    fp8_peak_sus = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+    warmup = max(3, args.warmup)
+    clocks = ClockSampler(local_rank)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------------------------------------------------------- decode set
+    xs_host, ws_host = decode_host_inputs()
+    qw_rot, sw_rot = {}, {}
+    for N, w in ws_host.items():
+        qw, sw = fp8bq.quantize_weight(w.to(dev))
+        qw_rot[N] = [qw] + [qw.clone() for _ in range(ROTATE - 1)]
+        sw_rot[N] = [sw] + [sw.clone() for _ in range(ROTATE - 1)]
+    calls = []
+    for g, xh in zip(W.DECODE_SET, xs_host):
+        x = xh.to(dev)
+        qa, sa = fp8bq.quantize_act(x)
+        calls.append({
+            "g": g, "x": x, "qa": qa, "sa": sa,
+            "y": torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev),
+            "ws_lin": fp8bq.new_workspace(fp8bq.OP_LINEAR, g.M, g.N, g.K, dev),
+            "ws_gemm": fp8bq.new_workspace(fp8bq.OP_GEMM, g.M, g.N, g.K, dev),
+            "x_pin": xh.pin_memory(),
+            "y_pin": torch.empty((g.M, g.N), dtype=torch.bfloat16).pin_memory(),
+        })
+    step_bytes = sum(linear_bytes(c["g"]) for c in calls)
+    gemm_step_bytes = sum(gemm_bytes(c["g"]) for c in calls)
+
+    def linear_step(r: int):
+        for c in calls:
+            N = c["g"].N
+            fp8bq.linear(c["x"], qw_rot[N][r], sw_rot[N][r], out=c["y"], workspace=c["ws_lin"])
+
+    def gemm_step(r: int):
+        for c in calls:
+            N = c["g"].N
+            fp8bq.gemm(c["qa"], c["sa"], qw_rot[N][r], sw_rot[N][r], out=c["y"],
+                       workspace=c["ws_gemm"])
+
+    # eager warm-up (also sets the library up on this device), launch counts per step
+    n0 = fp8bq.launch_count()
+    linear_step(0)
+    kernels_per_step = fp8bq.launch_count() - n0
+    n0 = fp8bq.launch_count()
+    gemm_step(0)
+    gemm_kernels_per_step = fp8bq.launch_count() - n0
+    torch.cuda.synchronize()
+
+    def capture(step_fn):
+        graphs = []
+        for r in range(ROTATE):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph):
+                step_fn(r)
+            graphs.append(gph)
+        return graphs
+
+    lin_graphs = capture(linear_step)
+    gemm_graphs = capture(gemm_step)
+    for i in range(warmup):
+        lin_graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+
+    barrier()
+    with clocks:
+        ms = events_ms(torch, lambda i: lin_graphs[i % ROTATE].replay(), args.steps)
+    barrier()
+    ms = max_over_ranks(ms)
+    value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9
+
+    # dominant kernel: the decode GEMM alone
+    for i in range(warmup):
+        gemm_graphs[i % ROTATE].replay()
+    barrier()
+    with clocks:
+        gms = events_ms(torch, lambda i: gemm_graphs[i % ROTATE].replay(), args.steps)
+    barrier()
+    gms = max_over_ranks(gms)
+    gemm_launches = args.steps * gemm_kernels_per_step
+    gemm_gbs = gemm_step_bytes * args.steps / (gms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": gemm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": None,
+                "kernel": "fp8bq::decode::gemm_decode_kernel",
+                "avg_launch_us": gms * 1e3 / gemm_launches,
+                "algorithmic_bytes_per_launch": gemm_step_bytes / gemm_kernels_per_step,
+                "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+
+    # ---------------------------------------------------------------- e2e through the API
+    def e2e_step(r: int):
+        for c in calls:
+            N = c["g"].N
+            c["x"].copy_(c["x_pin"], non_blocking=True)
+            fp8bq.linear(c["x"], qw_rot[N][r], sw_rot[N][r], out=c["y"], workspace=c["ws_lin"])
+            c["y_pin"].copy_(c["y"], non_blocking=True)
+
+    for i in range(warmup):
+        e2e_step(i % ROTATE)
+    barrier()
+    with clocks:
+        ems = events_ms(torch, lambda i: e2e_step(i % ROTATE), args.steps)
+    barrier()
+    ems = max_over_ranks(ems)
+    h2d = sum(c["g"].M * c["g"].K * 2 for c in calls)
+    d2h = sum(c["g"].M * c["g"].N * 2 for c in calls)
+    e2e = {"value": world * step_bytes * args.steps / (ems * 1e-3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "how": "per step and linear: pinned X -> device copy, fp8bq.linear, Y -> pinned "
+                  "host copy, eager launches from Python, CUDA events on the stream"}
+
+    extras = {}
+    if not args.quick:
+        extras = prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_sus,
+                                       args)
+
+    status = fp8bq.last_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the benchmark")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(xs_host, ws_host)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic (seeded numpy PCG64, BF16; weights quantized on the GPU)",
+            "config": {"workload": DECODE_WORKLOAD, "layers_per_step": len(calls),
+                       "algorithmic_bytes_per_step": step_bytes,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": f"inputs larger than L2: weights rotated over {ROTATE} device "
+                             "copies per shape",
+                       "timing": "CUDA events around CUDA-graph replays, max over ranks"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps * kernels_per_step,
+            "clocks": clocks.summary(),
+            "peaks": peaks,
+        }
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+
+
+def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_sus, args):
+    iters = max(5, min(20, args.steps))
+    warm = 3
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = {}
+
+    def shape_result(g: W.Gemm, with_linear: bool):
+        x = g.make_x().to(dev)
+        qw, sw = fp8bq.quantize_weight(g.make_w().to(dev))
+        qa, sa = fp8bq.quantize_act(x)
+        y = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
+        wsg = fp8bq.new_workspace(fp8bq.OP_GEMM, g.M, g.N, g.K, dev)
+        wsl = fp8bq.new_workspace(fp8bq.OP_LINEAR, g.M, g.N, g.K, dev)
+        with clocks:
+            tg = flushed_ms(torch, lambda: fp8bq.gemm(qa, sa, qw, sw, out=y, workspace=wsg),
+                            iters, warm, flush)
+            tl = flushed_ms(torch, lambda: fp8bq.linear(x, qw, sw, out=y, workspace=wsl),
+                            iters, warm, flush) if with_linear else None
+        r = {"name": g.name, "M": g.M, "N": g.N, "K": g.K}
+        mg = statistics.median(tg)
+        if g.M <= 16:
+            gbs = gemm_bytes(g) / (mg * 1e-3) / 1e9
+            r.update({"gemm_us": mg * 1e3, "gemm_gbs": gbs, "gemm_frac_hbm": gbs / peaks["hbm_gbs"]})
+            if tl:
+                ml = statistics.median(tl)
+                r.update({"linear_us": ml * 1e3,
+                          "linear_gbs": linear_bytes(g) / (ml * 1e-3) / 1e9})
+        else:
+            tf = g.flops / (mg * 1e-3) / 1e12
+            r.update({"gemm_us": mg * 1e3, "gemm_tflops": tf, "gemm_frac_fp8": tf / fp8_peak})
+            if tl:
+                ml = statistics.median(tl)
+                r.update({"linear_us": ml * 1e3, "linear_tflops": g.flops / (ml * 1e-3) / 1e12})
+        del x, qw, sw, qa, sa, y
+        return r
+
+    pq = shape_result(W.PREFILL_QKV, True)
+    out["prefill"] = {
+        "workload": "prefill fused QKV: X[8192,7168] x W[9216,7168]^T, BF16 out",
+        "metric": "TFLOP/s (2 M N K)", "linear_tflops": pq["linear_tflops"],
+        "linear_us": pq["linear_us"], "gemm_tflops": pq["gemm_tflops"],
+        "gemm_us": pq["gemm_us"],
+        "roofline": {"bound": "tensor", "achieved": pq["gemm_tflops"], "peak": fp8_peak,
+                     "unit": "TFLOP/s", "frac": pq["gemm_tflops"] / fp8_peak,
+                     "frac_of_sustained": pq["gemm_tflops"] / fp8_peak_sus, "traffic": None,
+                     "kernel": "fp8bq::prefill::gemm_prefill_kernel<256>",
+                     "peak_source": f"{peaks['source']} cuBLAS BF16 x 2 (nominal FP8/BF16 ratio)"},
+        "timing": f"median of {iters} launches, CUDA events, L2 flushed (256 MB write) before each",
+    }
+
+    # standalone activation quantizer on the long-prefill activation
+    g = W.LONG_O_PROJ
+    x = g.make_x().to(dev)
+    q = torch.empty((g.M, g.K), dtype=torch.uint8, device=dev)
+    s = torch.empty((g.M, g.K // 128), dtype=torch.float32, device=dev)
+    with clocks:
+        tq = flushed_ms(torch, lambda: fp8bq.quantize_act(x, q, s), iters, warm, flush)
+    mq = statistics.median(tq)
+    qbytes = g.M * g.K * 2 + g.M * g.K + g.M * (g.K // 128) * 4
+    out["quantize_act"] = {"shape": [g.M, g.K], "us": mq * 1e3, "gbs": qbytes / (mq * 1e-3) / 1e9,
+                           "frac_hbm": qbytes / (mq * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                           "algorithmic_bytes": qbytes}
+    del x, q, s
+
+    rows = [pq]
+    for g in (W.KPROJ_M16,) + W.DRAFTER_MLP + (W.LONG_O_PROJ,):
+        rows.append(shape_result(g, True))
+    out["workloads"] = rows
+    return out
+
+
+def cpu_baseline(xs_host, ws_host) -> dict:
+    import oracle
+    oracle.build()
+    qws = {N: oracle.quantize_weight(w) for N, w in ws_host.items()}   # offline step, untimed
+    secs, nbytes = oracle_decode_steps(oracle, xs_host, qws, 1)
+    steps = 1
+    while secs < 10.0 and steps < 16:
+        s2, b2 = oracle_decode_steps(oracle, xs_host, qws, 1)
+        secs += s2
+        nbytes += b2
+        steps += 1
+    return {"value": nbytes / secs / 1e9, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"{steps} full decode steps (the same 6 linears, all columns), "
+                      "oracle.linear_ref: plain C with OpenMP, FP64 GEMM accumulation"}
+
+
+def run_profile_case(case: str) -> None:
+    """A small, self-contained run of one kernel family (for ncu captures)."""
+    import torch
+
+    import fp8_block_scaled_09_b200 as fp8bq
+    dev = torch.device("cuda", 0)
+    t0 = time.perf_counter()
+    if case == "quantize":
+        g = W.LONG_O_PROJ
+        x = g.make_x().to(dev)
+        for _ in range(3):
+            fp8bq.quantize_act(x)
+    else:
+        gs = W.DECODE_SET if case == "decode" else (W.PREFILL_QKV,)
+        wq = {}
+        for g in gs:
+            if g.N not in wq:
+                wq[g.N] = fp8bq.quantize_weight(g.make_w().to(dev))
+        for g in gs:
+            x = g.make_x().to(dev)
+            qw, sw = wq[g.N]
+            qa, sa = fp8bq.quantize_act(x)
+            for _ in range(2):
+                fp8bq.gemm(qa, sa, qw, sw)
+                fp8bq.linear(x, qw, sw)
+    torch.cuda.synchronize()
+    status = fp8bq.last_device_status()
+    print(json.dumps({"profile_case": case, "launches": fp8bq.launch_count(), "status": status,
+                      "seconds": time.perf_counter() - t0}), flush=True)
+    if status != 0:
+        raise SystemExit(1)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--quick", action="store_true", help="decode set only (no prefill/workloads)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=("decode", "prefill", "quantize"),
+                    help="profiling case: run one kernel family a few times, print a short line")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if args.only:
+        run_profile_case(args.only)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -11,9 +11,11 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "fp8bq.h"
 #include "gemm_decode.cuh"
@@ -82,9 +84,16 @@ const DeviceInfo *device_info() {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  prefill::Layout<kPrefillBN>::kDynamicSmem) != cudaSuccess)
             return;
+        // The prefill kernel moves registers between warpgroups with setmaxnreg;
+        // the split is only safe if the launch allocates exactly what it was
+        // designed for (otherwise setmaxnreg.inc could wait forever).
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, prefill::gemm_prefill_kernel<kPrefillBN>) != cudaSuccess ||
+            fa.numRegs != prefill::kLaunchRegs)
+            return;
         if (cudaFuncSetAttribute(decode::gemm_decode_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode::Layout::kDynamicSmem) != cudaSuccess)
+                                 decode::Layout::kMaxSmem) != cudaSuccess)
             return;
         if (cudaDeviceSynchronize() != cudaSuccess) return;
         d.supported = true;
@@ -116,6 +125,28 @@ fp8bq_status check_mnk(int64_t M, int64_t N, int64_t K) {
 
 fp8bq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FP8BQ_OK : FP8BQ_ERR_CUDA; }
 
+// Every kernel is launched with programmatic stream serialization: it may be
+// scheduled while the previous kernel in the stream finishes, runs its
+// prologue (barrier set-up, TMEM allocation), and waits (griddepcontrol.wait)
+// before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+    return e;
+}
+
 // 2-D uint8 tensor map over a row-major [rows, cols] byte matrix, box
 // [box_rows, 128 bytes], 128-byte swizzle, zero fill out of bounds.
 bool make_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, uint32_t box_rows) {
@@ -134,8 +165,28 @@ bool make_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, ui
 
 size_t round256(int64_t b) { return static_cast<size_t>(((b + 255) / 256) * 256); }
 
+// The decode kernel takes M <= 16 as long as its staged scales fit in shared
+// memory (K up to roughly 1.6e5); anything else runs on the prefill kernel.
+// Decode grid: one CTA per SM, but at least kMinUnitsPerCta weight blocks per
+// CTA so small problems do not split every n-block across many CTAs.
+constexpr int64_t kMinUnitsPerCta = 4;
+int64_t decode_grid(int64_t units, int64_t sms) {
+    const int64_t by_work = (units + kMinUnitsPerCta - 1) / kMinUnitsPerCta;
+    return std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(sms, decode::kMaxGrid), by_work));
+}
+
+bool use_decode(int64_t M, int64_t N, int64_t K, int64_t sms) {
+    if (M > kDecodeMaxM || N / 128 > decode::kMaxCounters) return false;
+    const int64_t units = (N / 128) * (K / 128);
+    const int64_t grid = decode_grid(units, sms);
+    return decode::smem_bytes(K / 128, (units + grid - 1) / grid) <= decode::Layout::kMaxSmem;
+}
+
 size_t gemm_ws_bytes(int64_t M, int64_t N) {
-    if (M <= kDecodeMaxM) return round256(decode::workspace_bytes(N / 128));
+    // sized for the decode path whenever it may be chosen (the choice needs the
+    // device's SM count; the workspace does not depend on it)
+    if (M <= kDecodeMaxM && N / 128 <= decode::kMaxCounters)
+        return round256(decode::workspace_bytes(N / 128));
     return 0;
 }
 
@@ -150,17 +201,15 @@ cudaError_t launch_quantize_act(const DeviceInfo &d, const void *x, int64_t M, i
     const int64_t blocks_needed = (teams_needed * 16 + kActThreads - 1) / kActThreads;
     const int64_t max_blocks = static_cast<int64_t>(d.sm_count) * (2048 / kActThreads);
     const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
-    quantize_act_kernel<<<blocks, kActThreads, 0, st>>>(static_cast<const uint4 *>(x), groups,
-                                                       reinterpret_cast<uint2 *>(q), sa);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return cudaGetLastError();
+    return launch(quantize_act_kernel, dim3(blocks), dim3(kActThreads), 0, st,
+                  static_cast<const uint4 *>(x), groups, reinterpret_cast<uint2 *>(q), sa);
 }
 
 cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
                         const uint8_t *qw, const float *sw, int64_t M, int64_t N, int64_t K,
                         void *y, void *ws, cudaStream_t st, fp8bq_status *err) {
     *err = FP8BQ_OK;
-    if (M <= kDecodeMaxM) {
+    if (use_decode(M, N, K, d.sm_count)) {
         CUtensorMap tw, tx;
         if (!make_tmap(&tw, qw, N, K, decode::BNW) || !make_tmap(&tx, qa, M, K, decode::MT)) {
             *err = FP8BQ_ERR_CUDA;
@@ -168,16 +217,15 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
         }
         const int64_t NB = N / 128;
         const int64_t units = NB * (K / 128);
-        int64_t grid = d.sm_count;
-        if (grid > decode::kMaxGrid) grid = decode::kMaxGrid;
-        if (grid > units) grid = units;
+        const int64_t grid = decode_grid(units, d.sm_count);
         int *counters = static_cast<int *>(ws);
         float *partials =
-            reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::counters_bytes(NB));
-        decode::gemm_decode_kernel<<<static_cast<int>(grid), decode::kNumThreads,
-                                     decode::Layout::kDynamicSmem, st>>>(
-            tw, tx, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
-            static_cast<int>(N), static_cast<int>(K), counters, partials, d.status);
+            reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes);
+        const int64_t smem = decode::smem_bytes(K / 128, (units + grid - 1) / grid);
+        return launch(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(grid)),
+                      dim3(decode::kNumThreads), static_cast<size_t>(smem), st, tw, tx, sa, sw,
+                      static_cast<__nv_bfloat16 *>(y), static_cast<int>(M), static_cast<int>(N),
+                      static_cast<int>(K), counters, partials, d.status);
     } else {
         CUtensorMap ta, tb;
         if (!make_tmap(&ta, qa, M, K, prefill::BM) || !make_tmap(&tb, qw, N, K, kPrefillBN)) {
@@ -186,13 +234,11 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
         }
         const int64_t tiles = ((M + prefill::BM - 1) / prefill::BM) * ((N + kPrefillBN - 1) / kPrefillBN);
         const int grid = static_cast<int>(tiles < d.sm_count ? tiles : d.sm_count);
-        prefill::gemm_prefill_kernel<kPrefillBN>
-            <<<grid, prefill::kNumThreads, prefill::Layout<kPrefillBN>::kDynamicSmem, st>>>(
-                ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
-                static_cast<int>(N), static_cast<int>(K), d.status);
+        return launch(prefill::gemm_prefill_kernel<kPrefillBN>, dim3(grid),
+                      dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN>::kDynamicSmem, st,
+                      ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
+                      static_cast<int>(N), static_cast<int>(K), d.status);
     }
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return cudaGetLastError();
 }
 
 }  // namespace
@@ -226,10 +272,9 @@ fp8bq_status fp8bq_quantize_weight(const void *w_bf16, int64_t N, int64_t K, uin
     const DeviceInfo *d = device_info();
     if (!d) return FP8BQ_ERR_NO_DEVICE;
     const dim3 grid(static_cast<unsigned>(K / 128), static_cast<unsigned>(N / 128));
-    quantize_weight_kernel<<<grid, kWeightThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint16_t *>(w_bf16), K, q_e4m3, sw);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return from_cuda(cudaGetLastError());
+    return from_cuda(launch(quantize_weight_kernel, grid, dim3(kWeightThreads), 0,
+                            static_cast<cudaStream_t>(stream),
+                            static_cast<const uint16_t *>(w_bf16), K, q_e4m3, sw));
 }
 
 size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {

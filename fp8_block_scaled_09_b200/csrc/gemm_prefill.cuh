@@ -10,16 +10,19 @@
 // cannot carry, so every K chunk is a fresh tensor-core partial in TMEM that
 // CUDA cores promote into a register accumulator:  acc = fma(P_kb, sa*sw, acc).
 //
-// Design (one persistent CTA per SM, 320 threads):
+// Design (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warp 0      TMA producer: per K chunk one A tile (128 x 128 B) and one B tile
 //               (BN x 128 B), 128-byte swizzle, into a kStages-deep ring.
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 32 each) per chunk
 //               into one of two TMEM buffers of BN FP32 columns.
-//   warps 2..9  promotion + epilogue: warp w reads TMEM lanes 32*(w%4)..+31
-//               (its hardware lane quarter); warps 2-5 own tile columns
-//               [0, 128), warps 6-9 columns [128, 256), so each thread keeps the
-//               128 FP32 accumulators of one output row and one 128-column
-//               weight block, whose scale is a single sw value per chunk.
+//   warps 2-3   idle; warpgroup 0 gives its registers up (setmaxnreg 40).
+//   warps 4..11 promotion + epilogue (setmaxnreg 232): warp w reads TMEM lanes
+//               32*(w%4)..+31 (its hardware lane quarter); warpgroup 1 owns tile
+//               columns [0, 128), warpgroup 2 columns [128, 256), so a thread
+//               keeps the 128 FP32 accumulators of one output row in one
+//               128-column weight block, whose scale is a single sw per chunk.
+// Register budget: launched at 168 per thread (384 x 168 = 64512); after the
+// split 128 x 40 + 256 x 232 = 64512, the same total.
 // Tiles are walked in groups of kGroupM m-tiles so the tiles resident at one
 // time share A and B rows in L2.
 #pragma once
@@ -35,9 +38,16 @@ namespace prefill {
 constexpr int BM = 128;
 constexpr int BK = 128;  // one scale chunk of K per pipeline stage
 constexpr int kStages = 4;
-constexpr int kNumThreads = 320;
+constexpr int kNumThreads = 384;
+constexpr int kLaunchRegs = 168;     // registers per thread the kernel must be built with
+constexpr int kProducerRegs = 40;    // warpgroup 0 after setmaxnreg.dec
+constexpr int kConsumerRegs = 232;   // warpgroups 1-2 after setmaxnreg.inc
+static_assert(128 * kProducerRegs + 256 * kConsumerRegs <= kNumThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+constexpr int kFirstPromoWarp = 4;
 constexpr int kPromoWarps = 8;
 constexpr int kGroupM = 16;
+constexpr int kScaleLookahead = 2;   // K chunks of scale prefetch in registers
 
 template <int BN>
 struct Layout {
@@ -67,6 +77,152 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// Promotes one K chunk of this thread's 128 TMEM columns into acc:
+// acc[i] = fma(P[i], scale, acc[i]).  The four 32-column TMEM loads are
+// software-pipelined (the next load is in flight while the FMAs of the
+// current one run); the last chunk is returned in `last` after its wait, so
+// the caller can release the TMEM buffer before finishing its FMAs.  Loads and
+// waits live in one asm statement so no register is read before its wait.
+__device__ __forceinline__ void promote_chunk(uint32_t taddr, float scale, float (&acc)[128],
+                                              float (&last)[32]) {
+    asm volatile(
+        "{\n\t"
+        ".reg .f32 ra<32>, rb<32>;\n\t"
+        ".reg .b32 ta1, ta2, ta3;\n\t"
+        "add.u32 ta1, %129, 32;\n\t"
+        "add.u32 ta2, %129, 64;\n\t"
+        "add.u32 ta3, %129, 96;\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {ra0,ra1,ra2,ra3,ra4,ra5,ra6,ra7,ra8,ra9,ra10,ra11,ra12,ra13,ra14,ra15,ra16,ra17,ra18,ra19,ra20,ra21,ra22,ra23,ra24,ra25,ra26,ra27,ra28,ra29,ra30,ra31}, [%129];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {rb0,rb1,rb2,rb3,rb4,rb5,rb6,rb7,rb8,rb9,rb10,rb11,rb12,rb13,rb14,rb15,rb16,rb17,rb18,rb19,rb20,rb21,rb22,rb23,rb24,rb25,rb26,rb27,rb28,rb29,rb30,rb31}, [ta1];\n\t"
+        "fma.rn.f32 %0, ra0, %128, %0;\n\t"
+        "fma.rn.f32 %1, ra1, %128, %1;\n\t"
+        "fma.rn.f32 %2, ra2, %128, %2;\n\t"
+        "fma.rn.f32 %3, ra3, %128, %3;\n\t"
+        "fma.rn.f32 %4, ra4, %128, %4;\n\t"
+        "fma.rn.f32 %5, ra5, %128, %5;\n\t"
+        "fma.rn.f32 %6, ra6, %128, %6;\n\t"
+        "fma.rn.f32 %7, ra7, %128, %7;\n\t"
+        "fma.rn.f32 %8, ra8, %128, %8;\n\t"
+        "fma.rn.f32 %9, ra9, %128, %9;\n\t"
+        "fma.rn.f32 %10, ra10, %128, %10;\n\t"
+        "fma.rn.f32 %11, ra11, %128, %11;\n\t"
+        "fma.rn.f32 %12, ra12, %128, %12;\n\t"
+        "fma.rn.f32 %13, ra13, %128, %13;\n\t"
+        "fma.rn.f32 %14, ra14, %128, %14;\n\t"
+        "fma.rn.f32 %15, ra15, %128, %15;\n\t"
+        "fma.rn.f32 %16, ra16, %128, %16;\n\t"
+        "fma.rn.f32 %17, ra17, %128, %17;\n\t"
+        "fma.rn.f32 %18, ra18, %128, %18;\n\t"
+        "fma.rn.f32 %19, ra19, %128, %19;\n\t"
+        "fma.rn.f32 %20, ra20, %128, %20;\n\t"
+        "fma.rn.f32 %21, ra21, %128, %21;\n\t"
+        "fma.rn.f32 %22, ra22, %128, %22;\n\t"
+        "fma.rn.f32 %23, ra23, %128, %23;\n\t"
+        "fma.rn.f32 %24, ra24, %128, %24;\n\t"
+        "fma.rn.f32 %25, ra25, %128, %25;\n\t"
+        "fma.rn.f32 %26, ra26, %128, %26;\n\t"
+        "fma.rn.f32 %27, ra27, %128, %27;\n\t"
+        "fma.rn.f32 %28, ra28, %128, %28;\n\t"
+        "fma.rn.f32 %29, ra29, %128, %29;\n\t"
+        "fma.rn.f32 %30, ra30, %128, %30;\n\t"
+        "fma.rn.f32 %31, ra31, %128, %31;\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {ra0,ra1,ra2,ra3,ra4,ra5,ra6,ra7,ra8,ra9,ra10,ra11,ra12,ra13,ra14,ra15,ra16,ra17,ra18,ra19,ra20,ra21,ra22,ra23,ra24,ra25,ra26,ra27,ra28,ra29,ra30,ra31}, [ta2];\n\t"
+        "fma.rn.f32 %32, rb0, %128, %32;\n\t"
+        "fma.rn.f32 %33, rb1, %128, %33;\n\t"
+        "fma.rn.f32 %34, rb2, %128, %34;\n\t"
+        "fma.rn.f32 %35, rb3, %128, %35;\n\t"
+        "fma.rn.f32 %36, rb4, %128, %36;\n\t"
+        "fma.rn.f32 %37, rb5, %128, %37;\n\t"
+        "fma.rn.f32 %38, rb6, %128, %38;\n\t"
+        "fma.rn.f32 %39, rb7, %128, %39;\n\t"
+        "fma.rn.f32 %40, rb8, %128, %40;\n\t"
+        "fma.rn.f32 %41, rb9, %128, %41;\n\t"
+        "fma.rn.f32 %42, rb10, %128, %42;\n\t"
+        "fma.rn.f32 %43, rb11, %128, %43;\n\t"
+        "fma.rn.f32 %44, rb12, %128, %44;\n\t"
+        "fma.rn.f32 %45, rb13, %128, %45;\n\t"
+        "fma.rn.f32 %46, rb14, %128, %46;\n\t"
+        "fma.rn.f32 %47, rb15, %128, %47;\n\t"
+        "fma.rn.f32 %48, rb16, %128, %48;\n\t"
+        "fma.rn.f32 %49, rb17, %128, %49;\n\t"
+        "fma.rn.f32 %50, rb18, %128, %50;\n\t"
+        "fma.rn.f32 %51, rb19, %128, %51;\n\t"
+        "fma.rn.f32 %52, rb20, %128, %52;\n\t"
+        "fma.rn.f32 %53, rb21, %128, %53;\n\t"
+        "fma.rn.f32 %54, rb22, %128, %54;\n\t"
+        "fma.rn.f32 %55, rb23, %128, %55;\n\t"
+        "fma.rn.f32 %56, rb24, %128, %56;\n\t"
+        "fma.rn.f32 %57, rb25, %128, %57;\n\t"
+        "fma.rn.f32 %58, rb26, %128, %58;\n\t"
+        "fma.rn.f32 %59, rb27, %128, %59;\n\t"
+        "fma.rn.f32 %60, rb28, %128, %60;\n\t"
+        "fma.rn.f32 %61, rb29, %128, %61;\n\t"
+        "fma.rn.f32 %62, rb30, %128, %62;\n\t"
+        "fma.rn.f32 %63, rb31, %128, %63;\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [ta3];\n\t"
+        "fma.rn.f32 %64, ra0, %128, %64;\n\t"
+        "fma.rn.f32 %65, ra1, %128, %65;\n\t"
+        "fma.rn.f32 %66, ra2, %128, %66;\n\t"
+        "fma.rn.f32 %67, ra3, %128, %67;\n\t"
+        "fma.rn.f32 %68, ra4, %128, %68;\n\t"
+        "fma.rn.f32 %69, ra5, %128, %69;\n\t"
+        "fma.rn.f32 %70, ra6, %128, %70;\n\t"
+        "fma.rn.f32 %71, ra7, %128, %71;\n\t"
+        "fma.rn.f32 %72, ra8, %128, %72;\n\t"
+        "fma.rn.f32 %73, ra9, %128, %73;\n\t"
+        "fma.rn.f32 %74, ra10, %128, %74;\n\t"
+        "fma.rn.f32 %75, ra11, %128, %75;\n\t"
+        "fma.rn.f32 %76, ra12, %128, %76;\n\t"
+        "fma.rn.f32 %77, ra13, %128, %77;\n\t"
+        "fma.rn.f32 %78, ra14, %128, %78;\n\t"
+        "fma.rn.f32 %79, ra15, %128, %79;\n\t"
+        "fma.rn.f32 %80, ra16, %128, %80;\n\t"
+        "fma.rn.f32 %81, ra17, %128, %81;\n\t"
+        "fma.rn.f32 %82, ra18, %128, %82;\n\t"
+        "fma.rn.f32 %83, ra19, %128, %83;\n\t"
+        "fma.rn.f32 %84, ra20, %128, %84;\n\t"
+        "fma.rn.f32 %85, ra21, %128, %85;\n\t"
+        "fma.rn.f32 %86, ra22, %128, %86;\n\t"
+        "fma.rn.f32 %87, ra23, %128, %87;\n\t"
+        "fma.rn.f32 %88, ra24, %128, %88;\n\t"
+        "fma.rn.f32 %89, ra25, %128, %89;\n\t"
+        "fma.rn.f32 %90, ra26, %128, %90;\n\t"
+        "fma.rn.f32 %91, ra27, %128, %91;\n\t"
+        "fma.rn.f32 %92, ra28, %128, %92;\n\t"
+        "fma.rn.f32 %93, ra29, %128, %93;\n\t"
+        "fma.rn.f32 %94, ra30, %128, %94;\n\t"
+        "fma.rn.f32 %95, ra31, %128, %95;\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "}"
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+f"(acc[4]), "+f"(acc[5]),
+          "+f"(acc[6]), "+f"(acc[7]), "+f"(acc[8]), "+f"(acc[9]), "+f"(acc[10]), "+f"(acc[11]),
+          "+f"(acc[12]), "+f"(acc[13]), "+f"(acc[14]), "+f"(acc[15]), "+f"(acc[16]), "+f"(acc[17]),
+          "+f"(acc[18]), "+f"(acc[19]), "+f"(acc[20]), "+f"(acc[21]), "+f"(acc[22]), "+f"(acc[23]),
+          "+f"(acc[24]), "+f"(acc[25]), "+f"(acc[26]), "+f"(acc[27]), "+f"(acc[28]), "+f"(acc[29]),
+          "+f"(acc[30]), "+f"(acc[31]), "+f"(acc[32]), "+f"(acc[33]), "+f"(acc[34]), "+f"(acc[35]),
+          "+f"(acc[36]), "+f"(acc[37]), "+f"(acc[38]), "+f"(acc[39]), "+f"(acc[40]), "+f"(acc[41]),
+          "+f"(acc[42]), "+f"(acc[43]), "+f"(acc[44]), "+f"(acc[45]), "+f"(acc[46]), "+f"(acc[47]),
+          "+f"(acc[48]), "+f"(acc[49]), "+f"(acc[50]), "+f"(acc[51]), "+f"(acc[52]), "+f"(acc[53]),
+          "+f"(acc[54]), "+f"(acc[55]), "+f"(acc[56]), "+f"(acc[57]), "+f"(acc[58]), "+f"(acc[59]),
+          "+f"(acc[60]), "+f"(acc[61]), "+f"(acc[62]), "+f"(acc[63]), "+f"(acc[64]), "+f"(acc[65]),
+          "+f"(acc[66]), "+f"(acc[67]), "+f"(acc[68]), "+f"(acc[69]), "+f"(acc[70]), "+f"(acc[71]),
+          "+f"(acc[72]), "+f"(acc[73]), "+f"(acc[74]), "+f"(acc[75]), "+f"(acc[76]), "+f"(acc[77]),
+          "+f"(acc[78]), "+f"(acc[79]), "+f"(acc[80]), "+f"(acc[81]), "+f"(acc[82]), "+f"(acc[83]),
+          "+f"(acc[84]), "+f"(acc[85]), "+f"(acc[86]), "+f"(acc[87]), "+f"(acc[88]), "+f"(acc[89]),
+          "+f"(acc[90]), "+f"(acc[91]), "+f"(acc[92]), "+f"(acc[93]), "+f"(acc[94]), "+f"(acc[95]),
+          "=f"(last[0]), "=f"(last[1]), "=f"(last[2]), "=f"(last[3]), "=f"(last[4]), "=f"(last[5]),
+          "=f"(last[6]), "=f"(last[7]), "=f"(last[8]), "=f"(last[9]), "=f"(last[10]), "=f"(last[11]),
+          "=f"(last[12]), "=f"(last[13]), "=f"(last[14]), "=f"(last[15]), "=f"(last[16]),
+          "=f"(last[17]), "=f"(last[18]), "=f"(last[19]), "=f"(last[20]), "=f"(last[21]),
+          "=f"(last[22]), "=f"(last[23]), "=f"(last[24]), "=f"(last[25]), "=f"(last[26]),
+          "=f"(last[27]), "=f"(last[28]), "=f"(last[29]), "=f"(last[30]), "=f"(last[31])
+        : "f"(scale), "r"(taddr)
+        : "memory");
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kNumThreads, 1)
 gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -91,6 +247,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const int n_tiles = (N + BN - 1) / BN;
     const int num_tiles = m_tiles * n_tiles;
 
+    allow_dependent_launch();
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -114,77 +271,82 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
+    // Everything above overlaps the previous kernel in the stream; every global
+    // memory access below happens after it has completed.
+    grid_dependency_wait();
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            uint32_t stage = 0, phase = 0;
-            int64_t issued = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                int tm, tn;
-                tile_coords(t, m_tiles, n_tiles, tm, tn);
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *sa_tile = smem + stage * L::kStage;
-                    mbar_arrive_expect_tx(&full[stage], L::kStage);
-                    tma_load_2d(sa_tile, &tmap_a, &full[stage], kb * BK, tm * BM);
-                    tma_load_2d(sa_tile + L::kA, &tmap_b, &full[stage], kb * BK, tn * BN);
-                    ++issued;
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1;
+    if (warp < kFirstPromoWarp) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+        if (warp == 0) {
+            // ------------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                uint32_t stage = 0, phase = 0;
+                int64_t issued = 0;
+                bool ok = true;
+                for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                    int tm, tn;
+                    tile_coords(t, m_tiles, n_tiles, tm, tn);
+                    for (int kb = 0; kb < KB; ++kb) {
+                        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *st = smem + stage * L::kStage;
+                        mbar_arrive_expect_tx(&full[stage], L::kStage);
+                        tma_load_2d(st, &tmap_a, &full[stage], kb * BK, tm * BM);
+                        tma_load_2d(st + L::kA, &tmap_b, &full[stage], kb * BK, tn * BN);
+                        ++issued;
+                        if (++stage == kStages) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
                     }
                 }
+                // Before the CTA may exit, every load it issued must have landed.
+                for (int64_t i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+                    mbar_wait(&full[i % kStages], static_cast<uint32_t>((i / kStages) & 1), nullptr,
+                              status);
             }
-            // Before the CTA may exit, every load it issued must have landed.
-            for (int64_t i = (issued > kStages ? issued - kStages : 0); i < issued; ++i) {
-                const uint32_t s = static_cast<uint32_t>(i % kStages);
-                const uint32_t p = static_cast<uint32_t>((i / kStages) & 1);
-                mbar_wait(&full[s], p, nullptr, status);
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = umma_idesc_e4m3(BM, BN);
-            uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&tempty[buf], bphase ^ 1, abort_flag, status) ||
-                        !mbar_wait(&full[stage], phase, abort_flag, status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    const uint32_t a_addr = smem_addr(smem + stage * L::kStage);
-                    const uint32_t b_addr = a_addr + L::kA;
-                    const uint32_t d_tmem = tmem_base + buf * BN;
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                const uint32_t idesc = umma_idesc_e4m3(BM, BN);
+                uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
+                bool ok = true;
+                for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                    for (int kb = 0; kb < KB; ++kb) {
+                        if (!mbar_wait(&tempty[buf], bphase ^ 1, abort_flag, status) ||
+                            !mbar_wait(&full[stage], phase, abort_flag, status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint32_t a_addr = smem_addr(smem + stage * L::kStage);
+                        const uint32_t b_addr = a_addr + L::kA;
+                        const uint32_t d_tmem = tmem_base + buf * BN;
 #pragma unroll
-                    for (int j = 0; j < BK / 32; ++j)
-                        umma_e4m3(d_tmem, umma_desc_sw128(a_addr + 32 * j),
-                                  umma_desc_sw128(b_addr + 32 * j), idesc, j > 0 ? 1u : 0u);
-                    umma_commit(&empty[stage]);
-                    umma_commit(&tfull[buf]);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1;
+                        for (int j = 0; j < BK / 32; ++j)
+                            umma_e4m3(d_tmem, umma_desc_sw128(a_addr + 32 * j),
+                                      umma_desc_sw128(b_addr + 32 * j), idesc, j > 0 ? 1u : 0u);
+                        umma_commit(&empty[stage]);
+                        umma_commit(&tfull[buf]);
+                        if (++stage == kStages) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
+                        buf ^= 1;
+                        if (buf == 0) bphase ^= 1;
                     }
-                    buf ^= 1;
-                    if (buf == 0) bphase ^= 1;
                 }
+                // Wait for every MMA this thread issued before TMEM is released.
+                umma_commit(drain);
+                mbar_wait(drain, 0, nullptr, status);
             }
-            // Wait for every MMA this thread issued before TMEM is released.
-            umma_commit(drain);
-            mbar_wait(drain, 0, nullptr, status);
         }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
         // ------------------------------------------------------------ promotion + epilogue
-        const int pw = warp - 2;
+        const int pw = warp - kFirstPromoWarp;
         const int quarter = warp & 3;  // TMEM lane quarter accessible to this warp
         const int half = pw >> 2;      // which 128-column weight block of the tile
         const int row_in_tile = quarter * 32 + lane;
@@ -203,33 +365,42 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             float acc[128];
 #pragma unroll
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-            float sa_next = row_ok ? __ldg(sa_row) : 0.0f;
-            float sw_next = col_ok ? __ldg(sw_row) : 0.0f;
-            for (int kb = 0; kb < KB; ++kb) {
-                const float scale = sa_next * sw_next;
-                if (kb + 1 < KB) {
-                    sa_next = row_ok ? __ldg(sa_row + kb + 1) : 0.0f;
-                    sw_next = col_ok ? __ldg(sw_row + kb + 1) : 0.0f;
-                }
-                if (!mbar_wait(&tfull[buf], bphase, abort_flag, status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                       buf * BN + half * 128;
+            // scales of the next kScaleLookahead chunks, in a register ring
+            float sa_q[kScaleLookahead], sw_q[kScaleLookahead];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float v[16];
-                    tmem_load16(taddr + c * 16, v);
+            for (int j = 0; j < kScaleLookahead; ++j) {
+                sa_q[j] = (row_ok && j < KB) ? __ldg(sa_row + j) : 0.0f;
+                sw_q[j] = (col_ok && j < KB) ? __ldg(sw_row + j) : 0.0f;
+            }
+            for (int kb0 = 0; kb0 < KB && ok; kb0 += kScaleLookahead) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[c * 16 + i] = fmaf(v[i], scale, acc[c * 16 + i]);
+                for (int j = 0; j < kScaleLookahead; ++j) {
+                    const int kb = kb0 + j;
+                    if (kb >= KB) break;
+                    const float scale = sa_q[j] * sw_q[j];
+                    const int kn = kb + kScaleLookahead;
+                    if (kn < KB) {
+                        sa_q[j] = row_ok ? __ldg(sa_row + kn) : 0.0f;
+                        sw_q[j] = col_ok ? __ldg(sw_row + kn) : 0.0f;
+                    }
+                    if (!mbar_wait(&tfull[buf], bphase, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t taddr = tmem_base +
+                                           (static_cast<uint32_t>(quarter * 32) << 16) +
+                                           buf * BN + half * 128;
+                    float last[32];
+                    promote_chunk(taddr, scale, acc, last);
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[buf]);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(last[i], scale, acc[96 + i]);
+                    buf ^= 1;
+                    if (buf == 0) bphase ^= 1;
                 }
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[buf]);
-                buf ^= 1;
-                if (buf == 0) bphase ^= 1;
             }
             if (ok && row_ok && col_ok) {
                 uint4 *dst = reinterpret_cast<uint4 *>(y + static_cast<int64_t>(grow) * N + gcol);

@@ -65,6 +65,8 @@ constexpr int kActUnroll = 2;
 __global__ void __launch_bounds__(kActThreads)
 quantize_act_kernel(const uint4 *__restrict__ x, int64_t num_groups, uint2 *__restrict__ q,
                     float *__restrict__ sa) {
+    allow_dependent_launch();
+    grid_dependency_wait();
     const int sub = threadIdx.x & 15;  // lane within the 16-lane group team
     const int64_t team = (static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x) >> 4;
     const int64_t num_teams = (static_cast<int64_t>(gridDim.x) * kActThreads) >> 4;
@@ -108,6 +110,8 @@ __global__ void __launch_bounds__(kWeightThreads)
 quantize_weight_kernel(const uint16_t *__restrict__ w, int64_t K, uint8_t *__restrict__ q,
                        float *__restrict__ sw) {
     __shared__ uint32_t warp_max[kWeightThreads / 32];
+    allow_dependent_launch();
+    grid_dependency_wait();
     const int64_t bj = blockIdx.x;  // K block
     const int64_t bi = blockIdx.y;  // N block
     const int64_t KB = K / 128;

@@ -111,9 +111,10 @@ FP8BQ_API fp8bq_status fp8bq_quantize_weight(const void *w_bf16, int64_t N, int6
  *   y_bf16 : out, BF16 [M, N]
  *   workspace, ws_bytes : device scratch of at least
  *       fp8bq_workspace_size(FP8BQ_OP_GEMM, M, N, K) bytes (may be NULL when
- *       that is 0).  Its first fp8bq_workspace_size(...) bytes must hold the
- *       state left by fp8bq_workspace_init() or by a previous successful call;
- *       calls that share a workspace must be ordered (same stream).
+ *       that is 0).  Its contents must be the state left by
+ *       fp8bq_workspace_init() or by any previous successful fp8bq_gemm or
+ *       fp8bq_linear call, of any shape (every successful call restores that
+ *       state); calls that share a workspace must be ordered (same stream).
  * Output accuracy: |y - ref| <= 1e-2 |ref| + 2e-3 rms(ref) against the FP64 sum
  * of the dequantized operands; results are deterministic for a given shape.
  */

@@ -178,3 +178,41 @@ def test_linear_prefill_qkv_sampled():
     torch.cuda.synchronize()
     rows = sample_rows(g.M, 256, extra=(128, 4095, 4096))
     check(bf16_to_f64(y)[rows], oracle.linear_ref(x, qw, sw, rows=rows))
+
+
+def test_gemm_workspace_reused_across_calls():
+    # split-K counters must be back at zero after every call for the next one to be right
+    shapes = [(8, 9216, 7168), (16, 1024, 7168), (3, 16384, 256), (8, 9216, 7168)]
+    ws = torch.zeros(max(fp8bq.workspace_size(fp8bq.OP_GEMM, *s) for s in shapes),
+                     dtype=torch.uint8, device="cuda")
+    outs = []
+    for i, (M, N, K) in enumerate(shapes):
+        _, qa, sa, qw, sw = operands(M, N, K, 40 + (i % 3))
+        y = fp8bq.gemm(to_dev_codes(qa), to_dev_f32(sa), to_dev_codes(qw), to_dev_f32(sw),
+                       workspace=ws)
+        torch.cuda.synchronize()
+        check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
+        outs.append(y.cpu())
+    assert torch.equal(outs[0].view(torch.int16), outs[3].view(torch.int16))
+
+
+@pytest.mark.parametrize("M", [4, 333])
+def test_device_chain_without_host_sync(M):
+    # weight and activation quantization feed the GEMM on one stream with no host
+    # synchronization in between: each kernel must see its predecessor's output
+    N, K = 1152, 2048
+    x = workloads.activation(M, K, 77, outliers=3)
+    w = workloads.weight(N, K, 78)
+    xd, wd = x.cuda(), w.cuda()
+    torch.cuda.synchronize()
+    qw_d, sw_d = fp8bq.quantize_weight(wd)
+    qa_d, sa_d = fp8bq.quantize_act(xd)
+    y = fp8bq.gemm(qa_d, sa_d, qw_d, sw_d)
+    y2 = fp8bq.linear(xd, qw_d, sw_d)
+    torch.cuda.synchronize()
+    qw, sw = oracle.quantize_weight(w)
+    qa, sa = oracle.quantize_act(x)
+    assert np.array_equal(qw_d.cpu().numpy(), qw) and np.array_equal(qa_d.cpu().numpy(), qa)
+    ref = oracle.gemm_ref(qa, sa, qw, sw)
+    check(bf16_to_f64(y), ref)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
