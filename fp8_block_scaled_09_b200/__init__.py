@@ -23,7 +23,7 @@ import threading
 import torch
 
 __all__ = [
-    "Fp8bqError", "lib", "quantize_act", "quantize_weight", "gemm", "linear",
+    "Fp8bqError", "lib", "quantize_act", "quantize_weight", "gemm", "gemm_noalloc", "linear",
     "workspace_size", "new_workspace", "workspace_init", "last_device_status",
     "launch_count", "status_string", "OP_GEMM", "OP_LINEAR", "LIB_PATH",
 ]
@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_quantize_weight.argtypes = [P, I, I, P, P, P]
         L.fp8bq_gemm.argtypes = [P, P, P, P, I, I, I, P, P, S, P]
         L.fp8bq_linear.argtypes = [P, P, P, I, I, I, P, P, S, P]
+        L.fp8bq_gemm_noalloc.argtypes = [P, P, P, P, I, I, I, P, P]
         L.fp8bq_workspace_size.argtypes = [ctypes.c_int, I, I, I]
         L.fp8bq_workspace_size.restype = S
         L.fp8bq_workspace_init.argtypes = [P, S, P]
@@ -75,7 +76,7 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_version.argtypes = []
         L.fp8bq_version.restype = ctypes.c_int
         for name in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
-                     "fp8bq_workspace_init", "fp8bq_last_device_status"):
+                     "fp8bq_workspace_init", "fp8bq_last_device_status", "fp8bq_gemm_noalloc"):
             getattr(L, name).restype = st
         _lib = L
         return L
@@ -167,6 +168,24 @@ def gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
         workspace = new_workspace(OP_GEMM, M, N, K, qa.device)
     _check(lib().fp8bq_gemm(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), M, N, K, _ptr(out),
                             _ptr(workspace), workspace.numel(), _stream(qa)), "fp8bq_gemm")
+    return out
+
+
+def gemm_noalloc(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+                 out: torch.Tensor) -> torch.Tensor:
+    """fp8bq_gemm_noalloc: the GEMM with the library's built-in scratch instead of a
+    workspace, for callers that cannot allocate device memory.  `out` must be given
+    (this call allocates nothing); calls must not overlap on the GPU."""
+    qa, qw = _codes(qa), _codes(qw)
+    _need(qa, torch.uint8, "qa")
+    _need(qw, torch.uint8, "qw")
+    _need(sa, torch.float32, "sa")
+    _need(sw, torch.float32, "sw")
+    _need(out, torch.bfloat16, "out")
+    M, K = qa.shape
+    N = qw.shape[0]
+    _check(lib().fp8bq_gemm_noalloc(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), M, N, K, _ptr(out),
+                                    _stream(qa)), "fp8bq_gemm_noalloc")
     return out
 
 

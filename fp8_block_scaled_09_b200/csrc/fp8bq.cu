@@ -244,6 +244,20 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
 }  // namespace
 }  // namespace fp8bq
 
+// ---------------------------------------------------------------- allocation-free GEMM
+// Scratch for fp8bq_gemm_noalloc: a file-scope device array, so callers that
+// cannot allocate device memory need not supply a workspace.  Every GPU that
+// loads this library holds it until the process exits.
+namespace fp8bq {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+void *g_noalloc_ptr[kMaxDevices];
+cudaError_t g_noalloc_err[kMaxDevices];
+std::once_flag g_noalloc_once[kMaxDevices];
+}  // namespace
+}  // namespace fp8bq
+
 using namespace fp8bq;
 
 extern "C" {
@@ -367,5 +381,38 @@ const char *fp8bq_status_string(fp8bq_status status) {
 uint64_t fp8bq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int fp8bq_version(void) { return 100; }
+
+fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, const uint8_t *qw,
+                                const float *sw, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                                void *stream) {
+    fp8bq_status st = check_mnk(M, N, K);
+    if (st != FP8BQ_OK) return st;
+    if (M == 0) return FP8BQ_OK;
+    if (!qa || !sa || !qw || !sw || !y_bf16) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16))
+        return FP8BQ_ERR_MISALIGNED;
+    const size_t need = gemm_ws_bytes(M, N);
+    if (need > kNoAllocScratchBytes) return FP8BQ_ERR_WORKSPACE;  // beyond the built-in scratch
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP8BQ_ERR_CUDA;
+    // Once per device, with that device current: the array's device address.
+    // (In host code the array's name is only a host-side stand-in.)
+    std::call_once(g_noalloc_once[dev], [dev] {
+        g_noalloc_err[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+    });
+    if (g_noalloc_err[dev] != cudaSuccess || g_noalloc_ptr[dev] == nullptr) return FP8BQ_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // The array keeps whatever the previous call left; the split-K counters
+    // must start at zero, so clear them on this call's stream first.
+    if (need && cudaMemsetAsync(g_noalloc_ptr[dev], 0, static_cast<size_t>(decode::kCounterBytes),
+                                s) != cudaSuccess)
+        return FP8BQ_ERR_CUDA;
+    fp8bq_status err;
+    cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, g_noalloc_ptr[dev], s, &err);
+    if (err != FP8BQ_OK) return err;
+    return from_cuda(e);
+}
 
 }  // extern "C"

@@ -133,6 +133,27 @@ FP8BQ_API fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const
                           int64_t N, int64_t K, void *y_bf16, void *workspace, size_t ws_bytes,
                           void *stream);
 
+/*
+ * fp8bq_gemm without a workspace argument, for callers that cannot allocate
+ * device memory: code running where no allocator is reachable (an embedding
+ * runtime that hands out only fixed buffers, or a context where cudaMalloc is
+ * not permitted).  The paper has no counterpart; this is a convenience of the
+ * library.  Same arguments, results and accuracy as fp8bq_gemm, minus the
+ * workspace.  Its scratch is a 4 MiB array inside the library (held on every
+ * GPU that loads it until the process exits), so it rejects problems whose
+ * scratch would exceed that with FP8BQ_ERR_WORKSPACE: with M <= 16 that means
+ * N > 32512; larger M needs no scratch.  It calls no allocator.
+ *   - The first call on a device looks up the array's device address (a
+ *     one-time set-up); make that first call before any stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race and give wrong results; order them.
+ *   - Each call first clears the part of the array that must start at zero
+ *     (a memset on its stream).
+ */
+FP8BQ_API fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, const uint8_t *qw,
+                                          const float *sw, int64_t M, int64_t N, int64_t K,
+                                          void *y_bf16, void *stream);
+
 /* Bytes of workspace the operation needs for this shape (0 when none, and for
  * arguments the call would reject).  Always a multiple of 256. */
 FP8BQ_API size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K);
