@@ -50,6 +50,11 @@ import workloads as W  # noqa: E402
 METRIC = "FP8 block-scaled GEMM TFLOPS (prefill) & HBM GB/s (decode), % of roofline, 1 B200"
 FP8_OVER_BF16 = 2.0          # nominal dense ratio 4.5 / 2.25 PFLOP/s
 ROTATE = 4                   # device copies of each decode weight
+# DRAM bytes (read + write) of one decode GEMM launch, o_proj M=1 (7168 x 7168), from the ncu
+# capture summarised in profiles/gemm_decode_kernel_o_proj_m1.md; scaled to other shapes by
+# their algorithmic bytes (the capture shows DRAM bytes = algorithmic bytes within 0.04%).
+DECODE_TRAFFIC_CAPTURE = {"shape": (1, 7168, 7168), "dram_bytes": 51_441_664 + 4_096,
+                          "source": "profiles/gemm_decode_kernel_o_proj_m1.md"}
 DECODE_WORKLOAD = ("decode GEMV set: fp8bq_linear, M in {1,4,8} x {fused QKV W[9216,7168], "
                    "o_proj W[7168,7168]}, E4M3 128x128-blocked weights, X BF16 N(0,1) with "
                    "7 outlier channels x20")
@@ -336,8 +341,13 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     gms = max_over_ranks(gms)
     gemm_launches = args.steps * gemm_kernels_per_step
     gemm_gbs = gemm_step_bytes * args.steps / (gms * 1e-3) / 1e9
+    cap_M, cap_N, cap_K = DECODE_TRAFFIC_CAPTURE["shape"]
+    cap_ratio = DECODE_TRAFFIC_CAPTURE["dram_bytes"] / gemm_bytes(W.Gemm("capture", cap_M, cap_N, cap_K, 0))
+    traffic = cap_ratio * gemm_step_bytes / gemm_kernels_per_step
     roofline = {"bound": "hbm", "achieved": gemm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": None,
+                "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                "traffic_source": f"ncu dram read+write of one launch ({DECODE_TRAFFIC_CAPTURE['source']}),"
+                                  " scaled to this mix by algorithmic bytes",
                 "kernel": "fp8bq::decode::gemm_decode_kernel",
                 "avg_launch_us": gms * 1e3 / gemm_launches,
                 "algorithmic_bytes_per_launch": gemm_step_bytes / gemm_kernels_per_step,

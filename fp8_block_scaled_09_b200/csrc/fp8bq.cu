@@ -6,7 +6,8 @@
 //   quantize_act     -> quantize_act_kernel (HBM-bound, grid = k x SMs)
 //   quantize_weight  -> quantize_weight_kernel (one CTA per 128x128 block)
 //   gemm, M <= 16    -> decode::gemm_decode_kernel (stream-K over weight blocks)
-//   gemm, M > 16     -> prefill::gemm_prefill_kernel<256> (persistent tcgen05)
+//   gemm, 16 < M <= 128 -> prefill::gemm_prefill_kernel<256> (persistent tcgen05)
+//   gemm, M > 128    -> prefill2::gemm_prefill_pair_kernel (persistent, CTA pairs)
 //   linear           -> quantize_act into the workspace, then the gemm path
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -20,6 +21,7 @@
 #include "fp8bq.h"
 #include "gemm_decode.cuh"
 #include "gemm_prefill.cuh"
+#include "gemm_prefill2.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
 
@@ -33,12 +35,17 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kPrefillBN = 256;
+// The CTA-pair prefill kernel is correct but, with two 256-column TMEM buffers,
+// its cross-SM release round trip per K chunk leaves the tensor pipe idle more
+// than the single-CTA kernel; it stays off until it has deeper buffering.
+constexpr bool kUsePairPrefill = false;
 constexpr int64_t kDecodeMaxM = decode::MT;
 
 std::atomic<uint64_t> g_launches{0};
 
 struct DeviceInfo {
     int sm_count = 0;
+    int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair prefill kernel
     int *status = nullptr;  // device address of g_status
     bool supported = false;
 };
@@ -91,6 +98,31 @@ const DeviceInfo *device_info() {
         if (cudaFuncGetAttributes(&fa, prefill::gemm_prefill_kernel<kPrefillBN>) != cudaSuccess ||
             fa.numRegs != prefill::kLaunchRegs)
             return;
+        if (cudaFuncSetAttribute(prefill2::gemm_prefill_pair_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 prefill2::Layout::kDynamicSmem) != cudaSuccess)
+            return;
+        if (cudaFuncGetAttributes(&fa, prefill2::gemm_prefill_pair_kernel) != cudaSuccess ||
+            fa.numRegs != prefill2::kLaunchRegs)
+            return;
+        {
+            // how many 2-CTA clusters fit at once: the persistent pair grid size
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * (d.sm_count / 2));
+            cfg.blockDim = dim3(prefill2::kNumThreads);
+            cfg.dynamicSmemBytes = prefill2::Layout::kDynamicSmem;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = 2;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&d.pair_clusters, prefill2::gemm_prefill_pair_kernel,
+                                               &cfg) != cudaSuccess ||
+                d.pair_clusters < 1)
+                return;
+        }
         if (cudaFuncSetAttribute(decode::gemm_decode_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::Layout::kMaxSmem) != cudaSuccess)
@@ -130,21 +162,34 @@ fp8bq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FP8BQ_OK : FP8
 // prologue (barrier set-up, TMEM allocation), and waits (griddepcontrol.wait)
 // before touching global memory.
 template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                   Args &&...args) {
+cudaError_t launch_clustered(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, unsigned cluster_x, Args &&...args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cluster_x > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = cluster_x;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
     if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
     return e;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args &&...args) {
+    return launch_clustered(kernel, grid, block, smem, st, 1u, std::forward<Args>(args)...);
 }
 
 // 2-D uint8 tensor map over a row-major [rows, cols] byte matrix, box
@@ -226,6 +271,20 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
                       dim3(decode::kNumThreads), static_cast<size_t>(smem), st, tw, tx, sa, sw,
                       static_cast<__nv_bfloat16 *>(y), static_cast<int>(M), static_cast<int>(N),
                       static_cast<int>(K), counters, partials, d.status);
+    } else if (kUsePairPrefill && M > prefill::BM) {
+        // CTA pairs: each CTA loads 128 rows of A and 128 of the 256 weight rows
+        CUtensorMap ta, tb;
+        if (!make_tmap(&ta, qa, M, K, prefill2::kHalf) || !make_tmap(&tb, qw, N, K, prefill2::kHalf)) {
+            *err = FP8BQ_ERR_CUDA;
+            return cudaSuccess;
+        }
+        const int64_t tiles = ((M + prefill2::BM - 1) / prefill2::BM) *
+                              ((N + prefill2::BN - 1) / prefill2::BN);
+        const int64_t pairs = std::min<int64_t>(tiles, d.pair_clusters);
+        return launch_clustered(prefill2::gemm_prefill_pair_kernel, dim3(static_cast<unsigned>(2 * pairs)),
+                                dim3(prefill2::kNumThreads), prefill2::Layout::kDynamicSmem, st, 2u,
+                                ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
+                                static_cast<int>(N), static_cast<int>(K), d.status);
     } else {
         CUtensorMap ta, tb;
         if (!make_tmap(&ta, qa, M, K, prefill::BM) || !make_tmap(&tb, qw, N, K, kPrefillBN)) {
