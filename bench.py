@@ -153,6 +153,24 @@ class ClockSampler:
                 "source": "nvml, 2 ms polling during the timed regions"}
 
 
+def max_over_ranks(v: float, world: int, device=None) -> float:
+    """The largest value over all ranks (the timed region of the slowest replica)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, units_per_step: float, steps: int, ms_max: float,
+                       scale: float = 1e-9) -> float:
+    """Whole-job throughput of `world` replicas that each processed `units_per_step`
+    per step for `steps` steps, timed by the slowest one (weak scaling)."""
+    return world * units_per_step * steps / (ms_max * 1e-3) * scale
+
+
 def events_ms(torch, fn, iters: int) -> float:
     s = torch.cuda.current_stream()
     e0 = torch.cuda.Event(enable_timing=True)
@@ -260,12 +278,6 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # ---------------------------------------------------------------- decode set
     xs_host, ws_host = decode_host_inputs()
@@ -328,8 +340,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     with clocks:
         ms = events_ms(torch, lambda i: lin_graphs[i % ROTATE].replay(), args.steps)
     barrier()
-    ms = max_over_ranks(ms)
-    value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9
+    ms = max_over_ranks(ms, world, dev)
+    value = replica_throughput(world, step_bytes, args.steps, ms)
 
     # dominant kernel: the decode GEMM alone
     for i in range(warmup):
@@ -338,7 +350,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     with clocks:
         gms = events_ms(torch, lambda i: gemm_graphs[i % ROTATE].replay(), args.steps)
     barrier()
-    gms = max_over_ranks(gms)
+    gms = max_over_ranks(gms, world, dev)
     gemm_launches = args.steps * gemm_kernels_per_step
     gemm_gbs = gemm_step_bytes * args.steps / (gms * 1e-3) / 1e9
     cap_M, cap_N, cap_K = DECODE_TRAFFIC_CAPTURE["shape"]
@@ -367,10 +379,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     with clocks:
         ems = events_ms(torch, lambda i: e2e_step(i % ROTATE), args.steps)
     barrier()
-    ems = max_over_ranks(ems)
+    ems = max_over_ranks(ems, world, dev)
     h2d = sum(c["g"].M * c["g"].K * 2 for c in calls)
     d2h = sum(c["g"].M * c["g"].N * 2 for c in calls)
-    e2e = {"value": world * step_bytes * args.steps / (ems * 1e-3) / 1e9, "unit": "GB/s",
+    e2e = {"value": replica_throughput(world, step_bytes, args.steps, ems), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "how": "per step and linear: pinned X -> device copy, fp8bq.linear, Y -> pinned "
                   "host copy, eager launches from Python, CUDA events on the stream"}

@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "Fp8bqError", "lib", "quantize_act", "quantize_weight", "gemm", "gemm_noalloc", "linear",
     "workspace_size", "new_workspace", "workspace_init", "last_device_status",
-    "launch_count", "status_string", "OP_GEMM", "OP_LINEAR", "LIB_PATH",
+    "launch_count", "status_string", "selftest_timeout", "OP_GEMM", "OP_LINEAR", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bq.so")
@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_gemm.argtypes = [P, P, P, P, I, I, I, P, P, S, P]
         L.fp8bq_linear.argtypes = [P, P, P, I, I, I, P, P, S, P]
         L.fp8bq_gemm_noalloc.argtypes = [P, P, P, P, I, I, I, P, P]
+        L.fp8bq_selftest_timeout.argtypes = [ctypes.c_uint32, P]
         L.fp8bq_workspace_size.argtypes = [ctypes.c_int, I, I, I]
         L.fp8bq_workspace_size.restype = S
         L.fp8bq_workspace_init.argtypes = [P, S, P]
@@ -76,7 +77,8 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_version.argtypes = []
         L.fp8bq_version.restype = ctypes.c_int
         for name in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
-                     "fp8bq_workspace_init", "fp8bq_last_device_status", "fp8bq_gemm_noalloc"):
+                     "fp8bq_workspace_init", "fp8bq_last_device_status", "fp8bq_gemm_noalloc",
+                     "fp8bq_selftest_timeout"):
             getattr(L, name).restype = st
         _lib = L
         return L
@@ -211,6 +213,14 @@ def last_device_status(device=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     return int(lib().fp8bq_last_device_status(s))
+
+
+def selftest_timeout(limit_us: int = 20000) -> None:
+    """Enqueues the bounded-wait self-test (see fp8bq_selftest_timeout)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(lib().fp8bq_selftest_timeout(limit_us,
+                                        ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)),
+           "fp8bq_selftest_timeout")
 
 
 def launch_count() -> int:

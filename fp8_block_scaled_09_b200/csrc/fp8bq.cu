@@ -3,12 +3,14 @@
 //
 // All kernels live in this one translation unit so the device status word is a
 // single per-device symbol.  Dispatch:
-//   quantize_act     -> quantize_act_kernel (HBM-bound, grid = k x SMs)
+//   quantize_act     -> quantize_act_kernel (HBM-bound, persistent, bulk-copy ring)
 //   quantize_weight  -> quantize_weight_kernel (one CTA per 128x128 block)
 //   gemm, M <= 16    -> decode::gemm_decode_kernel (stream-K over weight blocks)
 //   gemm, 16 < M <= 128 -> prefill::gemm_prefill_kernel<256> (persistent tcgen05)
 //   gemm, M > 128    -> prefill2::gemm_prefill_pair_kernel (persistent, CTA pairs)
-//   linear           -> quantize_act into the workspace, then the gemm path
+//   linear           -> quantize_act into the workspace, then the gemm path; the
+//                       decode kernel then streams its first weight blocks while
+//                       the quantizer still runs (programmatic dependent launch)
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -30,6 +32,21 @@ namespace fp8bq {
 // Per-device status word: FP8BQ_OK or FP8BQ_ERR_TIMEOUT (set by a kernel that
 // abandoned a wait).  Read and cleared by fp8bq_last_device_status().
 __device__ int g_status;
+
+// Waits on a barrier that nothing ever arrives on: the bounded wait gives up
+// after limit_ns and records FP8BQ_ERR_TIMEOUT (exercises the failure path
+// every kernel uses, without faulting or hanging the GPU).
+__global__ void selftest_timeout_kernel(int *status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+}
 
 namespace {
 
@@ -98,14 +115,14 @@ const DeviceInfo *device_info() {
         if (cudaFuncGetAttributes(&fa, prefill::gemm_prefill_kernel<kPrefillBN>) != cudaSuccess ||
             fa.numRegs != prefill::kLaunchRegs)
             return;
-        if (cudaFuncSetAttribute(prefill2::gemm_prefill_pair_kernel,
+        // CTA-pair prefill kernel: optional; any failure here only leaves it off.
+        d.pair_clusters = 0;
+        if (kUsePairPrefill &&
+            cudaFuncSetAttribute(prefill2::gemm_prefill_pair_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 prefill2::Layout::kDynamicSmem) != cudaSuccess)
-            return;
-        if (cudaFuncGetAttributes(&fa, prefill2::gemm_prefill_pair_kernel) != cudaSuccess ||
-            fa.numRegs != prefill2::kLaunchRegs)
-            return;
-        {
+                                 prefill2::Layout::kDynamicSmem) == cudaSuccess &&
+            cudaFuncGetAttributes(&fa, prefill2::gemm_prefill_pair_kernel) == cudaSuccess &&
+            fa.numRegs == prefill2::kLaunchRegs) {
             // how many 2-CTA clusters fit at once: the persistent pair grid size
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(2 * (d.sm_count / 2));
@@ -119,10 +136,13 @@ const DeviceInfo *device_info() {
             cfg.attrs = at;
             cfg.numAttrs = 1;
             if (cudaOccupancyMaxActiveClusters(&d.pair_clusters, prefill2::gemm_prefill_pair_kernel,
-                                               &cfg) != cudaSuccess ||
-                d.pair_clusters < 1)
-                return;
+                                               &cfg) != cudaSuccess)
+                d.pair_clusters = 0;
+            cudaGetLastError();  // clear a failed query
         }
+        if (cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 ActLayout::kBytes) != cudaSuccess)
+            return;
         if (cudaFuncSetAttribute(decode::gemm_decode_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::Layout::kMaxSmem) != cudaSuccess)
@@ -242,17 +262,21 @@ size_t act_ws_bytes(int64_t M, int64_t K) { return round256(M * K) + round256(M 
 cudaError_t launch_quantize_act(const DeviceInfo &d, const void *x, int64_t M, int64_t K,
                                 uint8_t *q, float *sa, cudaStream_t st) {
     const int64_t groups = M * (K / 128);
-    const int64_t teams_needed = (groups + kActUnroll - 1) / kActUnroll;
-    const int64_t blocks_needed = (teams_needed * 16 + kActThreads - 1) / kActThreads;
-    const int64_t max_blocks = static_cast<int64_t>(d.sm_count) * (2048 / kActThreads);
-    const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
-    return launch(quantize_act_kernel, dim3(blocks), dim3(kActThreads), 0, st,
-                  static_cast<const uint4 *>(x), groups, reinterpret_cast<uint2 *>(q), sa);
+    const int64_t chunks = (groups + kActChunkGroups - 1) / kActChunkGroups;
+    const int64_t max_ctas = static_cast<int64_t>(d.sm_count) * kActCtasPerSm;
+    const int blocks = static_cast<int>(std::min(chunks, max_ctas));
+    return launch(quantize_act_kernel, dim3(blocks), dim3(kActThreads), ActLayout::kBytes, st,
+                  static_cast<const uint8_t *>(x), groups, reinterpret_cast<uint2 *>(q), sa,
+                  d.status);
 }
 
+// early_weights: the decode kernel may request its first weight blocks before
+// its dependency wait (only valid right after this library's activation
+// quantizer, see gemm_decode.cuh).
 cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
                         const uint8_t *qw, const float *sw, int64_t M, int64_t N, int64_t K,
-                        void *y, void *ws, cudaStream_t st, fp8bq_status *err) {
+                        void *y, void *ws, cudaStream_t st, fp8bq_status *err,
+                        bool early_weights = false) {
     *err = FP8BQ_OK;
     if (use_decode(M, N, K, d.sm_count)) {
         CUtensorMap tw, tx;
@@ -270,8 +294,8 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
         return launch(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(grid)),
                       dim3(decode::kNumThreads), static_cast<size_t>(smem), st, tw, tx, sa, sw,
                       static_cast<__nv_bfloat16 *>(y), static_cast<int>(M), static_cast<int>(N),
-                      static_cast<int>(K), counters, partials, d.status);
-    } else if (kUsePairPrefill && M > prefill::BM) {
+                      static_cast<int>(K), counters, partials, d.status, early_weights ? 1 : 0);
+    } else if (kUsePairPrefill && d.pair_clusters > 0 && M > prefill::BM) {
         // CTA pairs: each CTA loads 128 rows of A and 128 of the 256 weight rows
         CUtensorMap ta, tb;
         if (!make_tmap(&ta, qa, M, K, prefill2::kHalf) || !make_tmap(&tb, qw, N, K, prefill2::kHalf)) {
@@ -400,7 +424,7 @@ fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const float *sw
     cudaError_t e = launch_quantize_act(*d, x_bf16, M, K, qa, sa, s);
     if (e != cudaSuccess) return FP8BQ_ERR_CUDA;
     fp8bq_status err;
-    e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, gemm_ws, s, &err);
+    e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, gemm_ws, s, &err, /*early_weights=*/true);
     if (err != FP8BQ_OK) return err;
     return from_cuda(e);
 }
@@ -440,6 +464,16 @@ const char *fp8bq_status_string(fp8bq_status status) {
 uint64_t fp8bq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int fp8bq_version(void) { return 100; }
+
+fp8bq_status fp8bq_selftest_timeout(uint32_t limit_us, void *stream) {
+    if (limit_us == 0 || limit_us > 2000000u) return FP8BQ_ERR_INVALID_ARG;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        d->status, static_cast<uint64_t>(limit_us) * 1000u);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return from_cuda(cudaGetLastError());
+}
 
 fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, const uint8_t *qw,
                                 const float *sw, int64_t M, int64_t N, int64_t K, void *y_bf16,

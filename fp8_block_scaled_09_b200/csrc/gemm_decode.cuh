@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_x, const float *__restrict__ sa,
                    const float *__restrict__ sw, __nv_bfloat16 *__restrict__ y, int M, int N,
-                   int K, int *counters, float *partials, int *status) {
+                   int K, int *counters, float *partials, int *status, int early_weights) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -154,16 +154,35 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
-    // Everything above overlaps the previous kernel in the stream; every global
-    // memory access below happens after it has completed.
+    // Everything above overlaps the previous kernel in the stream.  With
+    // early_weights the first kStages weight blocks are requested too: only
+    // the linear layer sets it, when the previous kernel is its own activation
+    // quantizer, which writes activation codes and scales only and lets this
+    // kernel start after its own dependency wait.  Every other global access
+    // happens after the previous kernel has completed.
+    int64_t n_early = 0;
+    if (early_weights && warp == 0 && lane == 0) {
+        const uint64_t evict_first = l2_policy_evict_first();
+        for (int64_t u = u_begin; u < u_end && n_early < kStages; ++u, ++n_early) {
+            const int nb = static_cast<int>(u / KB), kb = static_cast<int>(u % KB);
+            mbar_arrive_expect_tx(&full[n_early], Layout::kStage);
+            tma_load_2d_hint(smem + n_early * Layout::kStage, &tmap_w, &full[n_early], kb * BK,
+                             nb * BNW, evict_first);
+        }
+    }
     grid_dependency_wait();
 
     if (warp == 0) {
         if (lane == 0) {
+            // activation tiles of the stages whose weight blocks went out early
+            for (int64_t i = 0; i < n_early; ++i)
+                tma_load_2d(smem + i * Layout::kStage + Layout::kW, &tmap_x, &full[i],
+                            static_cast<int>((u_begin + i) % KB) * BK, 0);
             const uint64_t evict_first = l2_policy_evict_first();
-            uint32_t stage = 0, phase = 0;
-            int64_t issued = 0;
-            for (int64_t u = u_begin; u < u_end; ++u) {
+            uint32_t stage = static_cast<uint32_t>(n_early % kStages);
+            uint32_t phase = n_early == kStages ? 1u : 0u;
+            int64_t issued = n_early;
+            for (int64_t u = u_begin + n_early; u < u_end; ++u) {
                 const int nb = static_cast<int>(u / KB), kb = static_cast<int>(u % KB);
                 if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) break;
                 uint8_t *st = smem + stage * Layout::kStage;

@@ -27,20 +27,19 @@ __device__ __forceinline__ float scale_from_amax_bits(uint32_t amax_bits) {
     return amax_bits == 0 ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax_bits), 448.0f);
 }
 
-// Eight BF16 values (one 16-byte vector) -> eight E4M3 codes (8 bytes).
+// Eight BF16 values (one 16-byte vector) -> eight E4M3 codes (8 bytes): each
+// code is the saturating round-to-nearest conversion of the IEEE quotient
+// fl32(x / scale).  (Division-free schemes that reproduce these codes exactly
+// -- a reciprocal with a rounding-interval check -- were measured and were
+// slower here than __fdiv_rn.)
 __device__ __forceinline__ uint2 encode8(uint4 v, float scale) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t out[2];
+    uint32_t c[4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const float a0 = __fdiv_rn(bf16_bits_to_float(w[2 * h] & 0xFFFFu), scale);
-        const float a1 = __fdiv_rn(bf16_bits_to_float(w[2 * h] >> 16), scale);
-        const float a2 = __fdiv_rn(bf16_bits_to_float(w[2 * h + 1] & 0xFFFFu), scale);
-        const float a3 = __fdiv_rn(bf16_bits_to_float(w[2 * h + 1] >> 16), scale);
-        out[h] = static_cast<uint32_t>(e4m3x2_satfinite(a0, a1)) |
-                 (static_cast<uint32_t>(e4m3x2_satfinite(a2, a3)) << 16);
-    }
-    return make_uint2(out[0], out[1]);
+    for (int i = 0; i < 4; ++i)
+        c[i] = e4m3x2_satfinite(__fdiv_rn(__uint_as_float(w[i] << 16), scale),
+                                __fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), scale));
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
 __device__ __forceinline__ uint32_t amax_bits8(uint4 v) {
@@ -56,46 +55,96 @@ __device__ __forceinline__ uint32_t amax_bits8(uint4 v) {
 
 // ------------------------------------------------------------------ activations
 
-// One 128-element group is handled by 16 consecutive lanes, each holding one
-// 16-byte vector (8 BF16).  Each thread takes kActUnroll groups per pass so
-// that several independent loads are in flight.
-constexpr int kActThreads = 256;
-constexpr int kActUnroll = 2;
+// The activation [M, K] is a flat sequence of M K / 128 groups of 256 bytes
+// (group g = row g / (K/128), channels 128 (g mod K/128) ...).  Persistent CTAs
+// (two per SM) stream chunks of kActChunkGroups groups through a kActStages-deep
+// shared-memory ring with untiled bulk copies, so the bytes in flight do not
+// depend on registers; sixteen consumer warps encode from shared memory, one
+// 16-lane team per group (one 16-byte vector per lane), and store codes and
+// scales straight to global memory.
+constexpr int kActConsumerWarps = 16;
+constexpr int kActThreads = 32 * (kActConsumerWarps + 1);  // + one producer warp
+constexpr int kActChunkGroups = 64;                         // 16 KB of BF16 per chunk
+constexpr int kActChunkBytes = kActChunkGroups * 256;
+constexpr int kActStages = 6;
+constexpr int kActCtasPerSm = 2;
 
-__global__ void __launch_bounds__(kActThreads)
-quantize_act_kernel(const uint4 *__restrict__ x, int64_t num_groups, uint2 *__restrict__ q,
-                    float *__restrict__ sa) {
-    allow_dependent_launch();
-    grid_dependency_wait();
-    const int sub = threadIdx.x & 15;  // lane within the 16-lane group team
-    const int64_t team = (static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x) >> 4;
-    const int64_t num_teams = (static_cast<int64_t>(gridDim.x) * kActThreads) >> 4;
+struct ActLayout {
+    static constexpr int kBarOff = kActStages * kActChunkBytes;
+    static constexpr int kBytes = kBarOff + 2 * kActStages * 8 + 16;
+};
 
-    // The loop bound uses the warp's first team so both teams of a warp iterate
-    // together (the shuffles below use the full warp mask).
-    const int64_t warp_team = team & ~static_cast<int64_t>(1);
-    for (int64_t it = warp_team; it < num_groups; it += num_teams * kActUnroll) {
-        const int64_t g0 = it + (team & 1);
-        uint4 v[kActUnroll];
-        bool ok[kActUnroll];
-#pragma unroll
-        for (int u = 0; u < kActUnroll; ++u) {
-            const int64_t g = g0 + u * num_teams;
-            ok[u] = g < num_groups;
-            v[u] = ok[u] ? __ldcs(x + g * 16 + sub) : make_uint4(0, 0, 0, 0);
+__global__ void __launch_bounds__(kActThreads, kActCtasPerSm)
+quantize_act_kernel(const uint8_t *__restrict__ x, int64_t num_groups, uint2 *__restrict__ q,
+                    float *__restrict__ sa, int *status) {
+    extern __shared__ __align__(128) uint8_t act_smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(act_smem + ActLayout::kBarOff);
+    uint64_t *empty = full + kActStages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kActStages);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t num_chunks = (num_groups + kActChunkGroups - 1) / kActChunkGroups;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kActStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kActConsumerWarps);
         }
-#pragma unroll
-        for (int u = 0; u < kActUnroll; ++u) {
-            uint32_t m = amax_bits8(v[u]);
-            // reduce over the 16 lanes of the team (xor offsets < 16 stay inside it)
-#pragma unroll
-            for (int off = 8; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-            const float scale = scale_from_amax_bits(m);
-            if (ok[u]) {
-                const int64_t g = g0 + u * num_teams;
-                q[g * 16 + sub] = encode8(v[u], scale);
-                if (sub == 0) sa[g] = scale;
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    grid_dependency_wait();
+    // The next kernel may start only once this one has passed its own wait: a
+    // GEMM that streams weights early then never overtakes the kernel that
+    // may have produced them.
+    allow_dependent_launch();
+
+    if (warp == kActConsumerWarps) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t evict_first = l2_policy_evict_first();
+            int64_t i = 0;
+            for (int64_t c = blockIdx.x; c < num_chunks; c += gridDim.x, ++i) {
+                const int s = static_cast<int>(i % kActStages);
+                if (!mbar_wait(&empty[s], static_cast<uint32_t>(((i / kActStages) & 1) ^ 1),
+                               abort_flag, status))
+                    break;
+                const int64_t g0 = c * kActChunkGroups;
+                const int64_t left = num_groups - g0;
+                const int64_t ng = left < kActChunkGroups ? left : kActChunkGroups;
+                const uint32_t bytes = static_cast<uint32_t>(ng * 256);
+                mbar_arrive_expect_tx(&full[s], bytes);
+                bulk_load(act_smem + s * kActChunkBytes, x + g0 * 256, bytes, &full[s], evict_first);
             }
+        }
+    } else {
+        // ------------------------------------------------------------ consumers
+        const int team = threadIdx.x >> 4;  // 0..31
+        const int sub = threadIdx.x & 15;
+        int64_t i = 0;
+        for (int64_t c = blockIdx.x; c < num_chunks; c += gridDim.x, ++i) {
+            const int s = static_cast<int>(i % kActStages);
+            if (!mbar_wait(&full[s], static_cast<uint32_t>((i / kActStages) & 1), abort_flag, status))
+                break;
+            const int64_t g0 = c * kActChunkGroups;
+            const uint8_t *st = act_smem + s * kActChunkBytes;
+#pragma unroll
+            for (int j = 0; j < kActChunkGroups / 32; ++j) {
+                const int gl = team + 32 * j;  // group within the chunk
+                const bool ok = g0 + gl < num_groups;
+                const uint4 v = ok ? *reinterpret_cast<const uint4 *>(st + gl * 256 + sub * 16)
+                                   : make_uint4(0, 0, 0, 0);
+                uint32_t m = amax_bits8(v);
+#pragma unroll
+                for (int off = 8; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+                const float scale = scale_from_amax_bits(m);
+                if (ok) {
+                    q[(g0 + gl) * 16 + sub] = encode8(v, scale);
+                    if (sub == 0) sa[g0 + gl] = scale;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
     }
 }

@@ -171,6 +171,13 @@ FP8BQ_API fp8bq_status fp8bq_last_device_status(void *stream);
 /* Static description of a status code (never NULL). */
 FP8BQ_API const char *fp8bq_status_string(fp8bq_status status);
 
+/* Diagnostic for the failure path: launches a kernel whose only internal wait
+ * can never complete, with the same bounded wait every kernel of the library
+ * uses, limited to limit_us microseconds (1 .. 2e6).  It returns after
+ * enqueueing; afterwards fp8bq_last_device_status() reports FP8BQ_ERR_TIMEOUT
+ * (and clears it).  Nothing faults or hangs; the context stays usable. */
+FP8BQ_API fp8bq_status fp8bq_selftest_timeout(uint32_t limit_us, void *stream);
+
 /* Number of kernels this library has launched in this process (all devices). */
 FP8BQ_API uint64_t fp8bq_launch_count(void);
 

@@ -146,6 +146,12 @@ def test_workspace_sizes(L):
 def test_valid_call_without_device_reports_no_device(L):
     assert L.fp8bq_quantize_act(GOOD, 4, 128, GOOD, GOOD, None) == NODEV
     assert L.fp8bq_last_device_status(None) == NODEV
+    assert L.fp8bq_selftest_timeout(20000, None) == NODEV
+
+
+def test_selftest_limit_is_validated_on_the_host(L):
+    assert L.fp8bq_selftest_timeout(0, None) == INVALID
+    assert L.fp8bq_selftest_timeout(2000001, None) == INVALID
 
 
 def test_binding_fails_loudly_without_cuda_tensors():

@@ -216,3 +216,21 @@ def test_device_chain_without_host_sync(M):
     ref = oracle.gemm_ref(qa, sa, qw, sw)
     check(bf16_to_f64(y), ref)
     assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+def test_decode_linear_near_ties_matches_unfused():
+    # activation rows whose quotients sit next to E4M3 rounding midpoints: the
+    # linear layer (quantizer + decode GEMM that streams weights early) must give
+    # a bit-identical output to quantize_act followed by gemm
+    from test_gpu_quantize import _near_tie_groups
+    x = _near_tie_groups()[:16].contiguous()
+    M, K = x.shape
+    w = workloads.weight(256, K, 91)
+    qw, sw = oracle.quantize_weight(w)
+    xd = x.cuda()
+    y = fp8bq.linear(xd, to_dev_codes(qw), to_dev_f32(sw))
+    qa, sa = fp8bq.quantize_act(xd)
+    y2 = fp8bq.gemm(qa, sa, to_dev_codes(qw), to_dev_f32(sw))
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    check(bf16_to_f64(y), oracle.linear_ref(x, qw, sw))

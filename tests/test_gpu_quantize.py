@@ -117,3 +117,31 @@ def test_quantize_weight_bit_exact(case):
 def test_quantize_weight_full_shapes(name):
     w = workloads.by_name(name).make_w()
     assert_same(gpu_quantize_weight(w), oracle.quantize_weight(w))
+
+
+def _near_tie_groups(n_scales=64, seed=3):
+    """Groups whose quotients x / s land within a few binary32 ulps of an E4M3
+    rounding midpoint (the quantizer's slowest and most fragile case)."""
+    rng = np.random.default_rng(seed)
+    all_bf16 = np.arange(0, 0x7F80, dtype=np.uint32)               # every finite positive BF16
+    xs = (all_bf16 << 16).view(np.float32)
+    rows = []
+    for _ in range(n_scales):
+        amax = np.float32(xs[rng.integers(0x3C00, 0x4700)])         # amax between ~2^-7 and ~2^15
+        s = np.float32(amax / np.float32(448.0))
+        cand = xs[xs <= amax]
+        t = (cand / s).astype(np.float32)
+        low = t.view(np.uint32) & 0xFFFFF
+        near = cand[(np.abs(low.astype(np.int64) - 0x80000) <= 12) & (t >= 2.0 ** -6)]
+        if near.size == 0:
+            continue
+        sign = np.where(rng.integers(0, 2, near.size) == 1, -1.0, 1.0).astype(np.float32)
+        vals = np.resize(near * sign, 127)
+        rows.append(np.concatenate([[amax], vals]).astype(np.float32))
+    assert len(rows) >= 16, "too few near-tie groups generated"
+    return _bf16(np.stack(rows))
+
+
+def test_quantize_act_near_e4m3_ties_bit_exact():
+    x = _near_tie_groups()
+    assert_same(gpu_quantize_act(x), oracle.quantize_act(x))
