@@ -185,19 +185,39 @@ def events_ms(torch, fn, iters: int) -> float:
 
 
 def flushed_ms(torch, fn, iters: int, warmup: int, flush) -> list[float]:
-    """Per-iteration event times with an L2 flush (untimed) before each iteration."""
+    """Per-iteration device times of fn with an L2 flush (untimed) before each.
+
+    fn is captured once into a CUDA graph and replayed, and a short device-side
+    sleep follows each flush, so the replay is already queued when the stream
+    reaches the start event: the interval holds the kernels only, not the
+    Python and driver time spent launching them.  The flush writes a buffer
+    larger than L2 and then reads it back, so L2 holds clean lines when the
+    timed kernels start (after a write alone, the kernels would pay for writing
+    back ~126 MB of the flush's dirty lines)."""
     s = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(s)
+    with torch.cuda.stream(side):
+        fn()
+    s.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fn()
+    torch.cuda.synchronize()
     evs = []
     for i in range(warmup + iters):
         flush.zero_()
+        flush.max()
+        torch.cuda._sleep(100_000)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(s)
-        fn()
+        graph.replay()
         e1.record(s)
         if i >= warmup:
             evs.append((e0, e1))
     torch.cuda.synchronize()
+    del graph
     return [a.elapsed_time(b) for a, b in evs]
 
 
@@ -442,19 +462,21 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
             tl = flushed_ms(torch, lambda: fp8bq.linear(x, qw, sw, out=y, workspace=wsl),
                             iters, warm, flush) if with_linear else None
         r = {"name": g.name, "M": g.M, "N": g.N, "K": g.K}
-        mg = statistics.median(tg)
-        if g.M <= 16:
+        mg = statistics.fmean(tg)
+        if g.M <= 128:
+            # weight-streaming regime (decode kernel): bandwidth is the bound
             gbs = gemm_bytes(g) / (mg * 1e-3) / 1e9
-            r.update({"gemm_us": mg * 1e3, "gemm_gbs": gbs, "gemm_frac_hbm": gbs / peaks["hbm_gbs"]})
+            r.update({"gemm_us": mg * 1e3, "gemm_gbs": gbs, "gemm_frac_hbm": gbs / peaks["hbm_gbs"],
+                      "gemm_tflops": g.flops / (mg * 1e-3) / 1e12})
             if tl:
-                ml = statistics.median(tl)
+                ml = statistics.fmean(tl)
                 r.update({"linear_us": ml * 1e3,
                           "linear_gbs": linear_bytes(g) / (ml * 1e-3) / 1e9})
         else:
             tf = g.flops / (mg * 1e-3) / 1e12
             r.update({"gemm_us": mg * 1e3, "gemm_tflops": tf, "gemm_frac_fp8": tf / fp8_peak})
             if tl:
-                ml = statistics.median(tl)
+                ml = statistics.fmean(tl)
                 r.update({"linear_us": ml * 1e3, "linear_tflops": g.flops / (ml * 1e-3) / 1e12})
         del x, qw, sw, qa, sa, y
         return r
@@ -470,7 +492,7 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
                      "frac_of_sustained": pq["gemm_tflops"] / fp8_peak_sus, "traffic": None,
                      "kernel": "fp8bq::prefill::gemm_prefill_kernel<256>",
                      "peak_source": f"{peaks['source']} cuBLAS BF16 x 2 (nominal FP8/BF16 ratio)"},
-        "timing": f"median of {iters} launches, CUDA events, L2 flushed (256 MB write) before each",
+        "timing": f"mean of {iters} graph replays, CUDA events, L2 flushed (256 MB write + read) before each",
     }
 
     # standalone activation quantizer on the long-prefill activation
@@ -480,12 +502,25 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
     s = torch.empty((g.M, g.K // 128), dtype=torch.float32, device=dev)
     with clocks:
         tq = flushed_ms(torch, lambda: fp8bq.quantize_act(x, q, s), iters, warm, flush)
-    mq = statistics.median(tq)
+    mq = statistics.fmean(tq)
     qbytes = g.M * g.K * 2 + g.M * g.K + g.M * (g.K // 128) * 4
     out["quantize_act"] = {"shape": [g.M, g.K], "us": mq * 1e3, "gbs": qbytes / (mq * 1e-3) / 1e9,
                            "frac_hbm": qbytes / (mq * 1e-3) / 1e9 / peaks["hbm_gbs"],
                            "algorithmic_bytes": qbytes}
     del x, q, s
+
+    mid = [shape_result(g, True) for g in W.MIDM_SET]
+    q128 = next(r for r in mid if r["name"] == "qkv_m128")
+    out["mid_m"] = {
+        "workload": "mid-size batches (32 and 128 rows) on fused QKV [9216,7168] and o_proj "
+                    "[7168,7168]: decode kernel with a 32- or 128-row token tile",
+        "rows": mid,
+        "roofline": {"bound": "hbm", "achieved": q128["gemm_gbs"], "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": q128["gemm_gbs"] / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "fp8bq::decode::gemm_decode_kernel<128> (qkv_m128)",
+                     "algorithmic_bytes": gemm_bytes(W.by_name("qkv_m128"))},
+        "timing": f"mean of {iters} graph replays, CUDA events, L2 flushed (256 MB write + read) before each",
+    }
 
     rows = [pq]
     for g in (W.KPROJ_M16,) + W.DRAFTER_MLP + (W.LONG_O_PROJ,):
@@ -524,7 +559,7 @@ def run_profile_case(case: str) -> None:
         for _ in range(3):
             fp8bq.quantize_act(x)
     else:
-        gs = W.DECODE_SET if case == "decode" else (W.PREFILL_QKV,)
+        gs = {"decode": W.DECODE_SET, "midm": W.MIDM_SET}.get(case, (W.PREFILL_QKV,))
         wq = {}
         for g in gs:
             if g.N not in wq:
@@ -552,7 +587,7 @@ def main() -> None:
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--quick", action="store_true", help="decode set only (no prefill/workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=("decode", "prefill", "quantize"),
+    ap.add_argument("--only", choices=("decode", "midm", "prefill", "quantize"),
                     help="profiling case: run one kernel family a few times, print a short line")
     args = ap.parse_args()
 

@@ -5,9 +5,10 @@
 // single per-device symbol.  Dispatch:
 //   quantize_act     -> quantize_act_kernel (HBM-bound, persistent, bulk-copy ring)
 //   quantize_weight  -> quantize_weight_kernel (one CTA per 128x128 block)
-//   gemm, M <= 16    -> decode::gemm_decode_kernel (stream-K over weight blocks)
-//   gemm, 16 < M <= 128 -> prefill::gemm_prefill_kernel<256> (persistent tcgen05)
-//   gemm, M > 128    -> prefill2::gemm_prefill_pair_kernel (persistent, CTA pairs)
+//   gemm, M <= 128   -> decode::gemm_decode_kernel<MT> (stream-K over weight
+//                       blocks; token tile MT = 16, 32, 64 or 128)
+//   gemm, M > 128    -> prefill::gemm_prefill_kernel<256> (persistent tcgen05;
+//                       the CTA-pair kernel prefill2 is built but not dispatched)
 //   linear           -> quantize_act into the workspace, then the gemm path; the
 //                       decode kernel then streams its first weight blocks while
 //                       the quantizer still runs (programmatic dependent launch)
@@ -56,7 +57,7 @@ constexpr int kPrefillBN = 256;
 // its cross-SM release round trip per K chunk leaves the tensor pipe idle more
 // than the single-CTA kernel; it stays off until it has deeper buffering.
 constexpr bool kUsePairPrefill = false;
-constexpr int64_t kDecodeMaxM = decode::MT;
+constexpr int64_t kDecodeMaxM = decode::kMaxMT;
 
 std::atomic<uint64_t> g_launches{0};
 
@@ -143,9 +144,18 @@ const DeviceInfo *device_info() {
         if (cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  ActLayout::kBytes) != cudaSuccess)
             return;
-        if (cudaFuncSetAttribute(decode::gemm_decode_kernel,
+        if (cudaFuncSetAttribute(decode::gemm_decode_kernel<16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode::Layout::kMaxSmem) != cudaSuccess)
+                                 decode::kMaxSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::gemm_decode_kernel<32>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::kMaxSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::gemm_decode_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::kMaxSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(decode::gemm_decode_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode::kMaxSmem) != cudaSuccess)
             return;
         if (cudaDeviceSynchronize() != cudaSuccess) return;
         d.supported = true;
@@ -230,8 +240,9 @@ bool make_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, ui
 
 size_t round256(int64_t b) { return static_cast<size_t>(((b + 255) / 256) * 256); }
 
-// The decode kernel takes M <= 16 as long as its staged scales fit in shared
-// memory (K up to roughly 1.6e5); anything else runs on the prefill kernel.
+// The decode kernel takes M <= 128 as long as its staged scales leave room for
+// at least kMinStages ring slots (for M <= 16, K up to roughly 1.4e5; for
+// M > 64, up to roughly 2.6e4); anything else runs on the prefill kernel.
 // Decode grid: one CTA per SM, but at least kMinUnitsPerCta weight blocks per
 // CTA so small problems do not split every n-block across many CTAs.
 constexpr int64_t kMinUnitsPerCta = 4;
@@ -240,18 +251,25 @@ int64_t decode_grid(int64_t units, int64_t sms) {
     return std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(sms, decode::kMaxGrid), by_work));
 }
 
-bool use_decode(int64_t M, int64_t N, int64_t K, int64_t sms) {
-    if (M > kDecodeMaxM || N / 128 > decode::kMaxCounters) return false;
+// Ring stages of the decode kernel for this shape, or 0 if it does not apply.
+int decode_stages(int64_t M, int64_t N, int64_t K, int64_t sms) {
+    if (M > kDecodeMaxM || N / 128 > decode::kMaxCounters) return 0;
     const int64_t units = (N / 128) * (K / 128);
     const int64_t grid = decode_grid(units, sms);
-    return decode::smem_bytes(K / 128, (units + grid - 1) / grid) <= decode::Layout::kMaxSmem;
+    const int64_t upc = (units + grid - 1) / grid, KB = K / 128;
+    switch (decode::token_tile(M)) {
+        case 16: return decode::pick_stages<16>(KB, upc);
+        case 32: return decode::pick_stages<32>(KB, upc);
+        case 64: return decode::pick_stages<64>(KB, upc);
+        default: return decode::pick_stages<128>(KB, upc);
+    }
 }
 
 size_t gemm_ws_bytes(int64_t M, int64_t N) {
     // sized for the decode path whenever it may be chosen (the choice needs the
     // device's SM count; the workspace does not depend on it)
     if (M <= kDecodeMaxM && N / 128 <= decode::kMaxCounters)
-        return round256(decode::workspace_bytes(N / 128));
+        return round256(decode::workspace_bytes(N / 128, decode::token_tile(M)));
     return 0;
 }
 
@@ -270,31 +288,47 @@ cudaError_t launch_quantize_act(const DeviceInfo &d, const void *x, int64_t M, i
                   d.status);
 }
 
+template <int MT>
+cudaError_t launch_decode(const DeviceInfo &d, const uint8_t *qa, const float *sa,
+                          const uint8_t *qw, const float *sw, int64_t M, int64_t N, int64_t K,
+                          void *y, void *ws, cudaStream_t st, fp8bq_status *err,
+                          bool early_weights, int stages) {
+    CUtensorMap tw, tx;
+    if (!make_tmap(&tw, qw, N, K, decode::BNW) || !make_tmap(&tx, qa, M, K, MT)) {
+        *err = FP8BQ_ERR_CUDA;
+        return cudaSuccess;
+    }
+    const int64_t units = (N / 128) * (K / 128);
+    const int64_t grid = decode_grid(units, d.sm_count);
+    int *counters = static_cast<int *>(ws);
+    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes);
+    const int64_t smem = decode::smem_bytes<MT>(stages, K / 128, (units + grid - 1) / grid);
+    return launch(decode::gemm_decode_kernel<MT>, dim3(static_cast<unsigned>(grid)),
+                  dim3(decode::Roles<MT>::kNumThreads), static_cast<size_t>(smem), st, tw, tx, sa, sw,
+                  static_cast<__nv_bfloat16 *>(y), static_cast<int>(M), static_cast<int>(N),
+                  static_cast<int>(K), counters, partials, d.status, early_weights ? 1 : 0,
+                  stages);
+}
+
 // early_weights: the decode kernel may request its first weight blocks before
 // its dependency wait (only valid right after this library's activation
 // quantizer, see gemm_decode.cuh).
 cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
                         const uint8_t *qw, const float *sw, int64_t M, int64_t N, int64_t K,
                         void *y, void *ws, cudaStream_t st, fp8bq_status *err,
-                        bool early_weights = false) {
+                        bool early_weights = false, bool allow_decode = true) {
     *err = FP8BQ_OK;
-    if (use_decode(M, N, K, d.sm_count)) {
-        CUtensorMap tw, tx;
-        if (!make_tmap(&tw, qw, N, K, decode::BNW) || !make_tmap(&tx, qa, M, K, decode::MT)) {
-            *err = FP8BQ_ERR_CUDA;
-            return cudaSuccess;
+    if (const int stages = allow_decode ? decode_stages(M, N, K, d.sm_count) : 0) {
+        switch (decode::token_tile(M)) {
+            case 16:
+                return launch_decode<16>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, stages);
+            case 32:
+                return launch_decode<32>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, stages);
+            case 64:
+                return launch_decode<64>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, stages);
+            default:
+                return launch_decode<128>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, stages);
         }
-        const int64_t NB = N / 128;
-        const int64_t units = NB * (K / 128);
-        const int64_t grid = decode_grid(units, d.sm_count);
-        int *counters = static_cast<int *>(ws);
-        float *partials =
-            reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes);
-        const int64_t smem = decode::smem_bytes(K / 128, (units + grid - 1) / grid);
-        return launch(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(grid)),
-                      dim3(decode::kNumThreads), static_cast<size_t>(smem), st, tw, tx, sa, sw,
-                      static_cast<__nv_bfloat16 *>(y), static_cast<int>(M), static_cast<int>(N),
-                      static_cast<int>(K), counters, partials, d.status, early_weights ? 1 : 0);
     } else if (kUsePairPrefill && d.pair_clusters > 0 && M > prefill::BM) {
         // CTA pairs: each CTA loads 128 rows of A and 128 of the 256 weight rows
         CUtensorMap ta, tb;
@@ -484,8 +518,12 @@ fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, const uint8_
     if (!qa || !sa || !qw || !sw || !y_bf16) return FP8BQ_ERR_INVALID_ARG;
     if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16))
         return FP8BQ_ERR_MISALIGNED;
-    const size_t need = gemm_ws_bytes(M, N);
-    if (need > kNoAllocScratchBytes) return FP8BQ_ERR_WORKSPACE;  // beyond the built-in scratch
+    size_t need = gemm_ws_bytes(M, N);
+    // Beyond the built-in scratch: M <= 16 is refused; larger M runs on the
+    // prefill kernel, which needs no scratch.
+    const bool fits = need <= kNoAllocScratchBytes;
+    if (!fits && M <= 16) return FP8BQ_ERR_WORKSPACE;
+    if (!fits) need = 0;
     const DeviceInfo *d = device_info();
     if (!d) return FP8BQ_ERR_NO_DEVICE;
     int dev = -1;
@@ -503,7 +541,8 @@ fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, const uint8_
                                 s) != cudaSuccess)
         return FP8BQ_ERR_CUDA;
     fp8bq_status err;
-    cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, g_noalloc_ptr[dev], s, &err);
+    cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, g_noalloc_ptr[dev], s, &err,
+                                /*early_weights=*/false, /*allow_decode=*/fits);
     if (err != FP8BQ_OK) return err;
     return from_cuda(e);
 }

@@ -1,22 +1,29 @@
-// gemm_decode.cuh -- block-scaled FP8 GEMM for small M (decode, M <= 16).
+// gemm_decode.cuh -- block-scaled FP8 GEMM for small M (decode and mid-size
+// batches, M <= 128), swap-AB and stream-K over the weight blocks.
 //
 // Same result as the prefill kernel (page "ProCreations/Nanbeige4.3-33B-FP8",
 // introduction: W8A8 FP8 linear layers), shaped for the weight-bandwidth-bound
 // regime: every weight byte is read from HBM exactly once, and the grid streams
 // the N/128 x K/128 weight blocks (16 KB each) evenly over all SMs.
 //
-// Roles (224 threads):
+// Roles (224 threads; 352 with eight promotion warps):
 //   warp 0      TMA producer: per unit (n-block nb, k-block kb) the 128 x 128 B
-//               weight block and the 16 x 128 B activation tile (rows >= M are
-//               zero-filled by TMA), kStages deep.
+//               weight block and the MT x 128 B activation tile (rows >= M are
+//               zero-filled by TMA).  Units travel in steps of kStep = 2: one
+//               ring slot, one full/empty barrier pair and one TMEM group per
+//               step, so the MMA thread touches shared memory (barrier waits)
+//               once per two units; each such access after issued MMAs costs
+//               it ~0.1 us, about the time a unit's data takes to arrive.
 //   warp 1      MMA issuer: swap-AB, D[n, m] = W_blk[n, :] . X_tile[m, :] with
-//               M_mma = 128 (weight rows) and N_mma = 16 (tokens), 4 MMAs of K = 32,
-//               into one of kTmemBufs TMEM buffers.
-//   warps 2..5  promotion: thread = one weight row n of the block (its TMEM
-//               lane), 16 FP32 accumulators (one per token); per unit
+//               M_mma = 128 (weight rows) and N_mma = MT (the token tile: 16,
+//               32, 64 or 128 rows, the smallest >= M), 4 MMAs of K = 32 per
+//               unit, each unit into its own TMEM slot.
+//   warps 2..   promotion (4 warps, or 8 from MT = 64): thread = one weight row
+//               n of the block (its TMEM lane) and MT or MT/2 token columns,
+//               one FP32 accumulator each; per unit
 //               acc[m] = fma(P[n, m], sa[m, kb] * sw[nb, kb], acc[m]), scales read
 //               from shared memory where they are staged once per CTA.
-//   warp 6      split-K: publishes this CTA's partial sums (device-wide fence and
+//   last warp   split-K: publishes this CTA's partial sums (device-wide fence and
 //               counter increment), so promotion never waits on either; if the
 //               CTA was an n-block's last contributor, all warps reduce it after
 //               the main loop.
@@ -39,30 +46,76 @@ namespace decode {
 
 constexpr int BNW = 128;  // weight rows per unit (one scale block)
 constexpr int BK = 128;
-constexpr int MT = 16;    // token tile (MMA N)
-constexpr int kStages = 8;
-constexpr int kNumThreads = 224;
-constexpr int kSplitWarp = 6;
-constexpr int kTmemBufs = 8;
-constexpr uint32_t kTmemCols = 128;  // kTmemBufs x MT columns
-constexpr int kMaxGrid = 256;        // workspace is sized for at most this many CTAs
+constexpr int kMaxMT = 128;
+constexpr int kMaxGrid = 256;  // workspace is sized for at most this many CTAs
 
-struct Layout {
-    static constexpr int kW = BNW * BK;  // 16 KB
-    static constexpr int kX = MT * BK;   // 2 KB
-    static constexpr int kStage = kW + kX;
-    static constexpr int kBarOff = kStages * kStage;
-    // full, empty (per stage), tfull, tempty (per TMEM buffer), drain, 2 split-K flushes
-    static constexpr int kNumBars = 2 * kStages + 2 * kTmemBufs + 1 + 2;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kScaleOff = kMiscOff + 16;  // then sa[MT][KB], then sw[units of this CTA]
-    static constexpr int kMaxSmem = 227 * 1024;
+// Warp roles for a token tile of MT rows: 4 promotion warps (one per TMEM lane
+// quarter) up to MT = 32, 8 from MT = 64 on (two per quarter, each owning half
+// of the token columns, so two warps per scheduler hide each other's TMEM and
+// shared-memory latency and each holds MT/2 accumulators).
+template <int MT>
+struct Roles {
+    static constexpr int kPromoWarps = MT >= 64 ? 8 : 4;
+    static constexpr int kPromoThreads = 32 * kPromoWarps;
+    static constexpr int kCols = MT * 4 / kPromoWarps;  // token columns per promotion thread
+    static constexpr int kSplitWarp = 2 + kPromoWarps;
+    static constexpr int kNumThreads = 32 * (kSplitWarp + 1);  // 224 or 352
 };
 
-// Dynamic shared memory for a launch: stages, barriers, the activation scales
-// of all M rows and the weight scales of one CTA's unit range.
-__host__ __device__ inline int64_t smem_bytes(int64_t KB, int64_t units_per_cta_max) {
-    return Layout::kScaleOff + MT * KB * 4 + (units_per_cta_max + 1) * 4 + 1024;
+// Smallest supported token tile holding M rows.
+__host__ __device__ constexpr int token_tile(int64_t M) {
+    return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+}
+
+// Units per ring slot / barrier / TMEM group, by token tile.
+__host__ __device__ constexpr int step_units_of(int /*MT*/) { return 2; }
+constexpr int kMaxRingUnits = 12;   // ring slots x units per slot, at most
+constexpr int kMinStages = 2;
+constexpr int kMaxSmem = 227 * 1024;
+
+// Shared memory: `stages` ring slots of kStep (weight block, activation tile), then
+// the barriers, a few words of CTA state, the activation scales [KB][MT + 4]
+// (transposed, so one thread reads four tokens' scales at once; the 4 extra
+// words per row make the transposing stores bank-conflict free) and the
+// weight scales of the CTA's unit range.  The stage count is chosen per launch
+// from what the scales leave of the 227 KB.
+template <int MT>
+struct Layout {
+    static_assert(MT == 16 || MT == 32 || MT == 64 || MT == 128, "token tile");
+    static constexpr int kStep = step_units_of(MT);
+    static constexpr int kMaxStages = kMaxRingUnits / kStep;
+    static constexpr int kTmemSlots = (512 / MT) < 8 ? (512 / MT) : 8;  // one unit each
+    static constexpr int kGroups = kTmemSlots / kStep;                   // one step each
+    static_assert(kGroups * kStep == kTmemSlots, "TMEM slots per group");
+    static constexpr uint32_t kTmemCols = static_cast<uint32_t>(kTmemSlots * MT);  // 128..512
+    static constexpr int kW = BNW * BK;  // 16 KB
+    static constexpr int kX = MT * BK;   // 2-16 KB
+    static constexpr int kUnit = kW + kX;
+    static constexpr int kStage = kStep * kUnit;
+    static constexpr int kSaRow = MT + 4;  // floats per staged activation-scale row
+    __host__ __device__ static constexpr int bar_off(int stages) { return stages * kStage; }
+    // full, empty (per stage), tfull, tempty (per TMEM group), drain, 2 split-K flushes
+    __host__ __device__ static constexpr int misc_off(int stages) {
+        return bar_off(stages) + (2 * stages + 2 * kGroups + 3) * 8;
+    }
+    __host__ __device__ static constexpr int scale_off(int stages) {
+        return (misc_off(stages) + 16 + 15) & ~15;  // float4 reads of the scales
+    }
+};
+
+// Dynamic shared memory for a launch (1 KB of it for the alignment of the ring).
+template <int MT>
+__host__ __device__ inline int64_t smem_bytes(int stages, int64_t KB, int64_t units_per_cta_max) {
+    return Layout<MT>::scale_off(stages) + Layout<MT>::kSaRow * KB * 4 + (units_per_cta_max + 1) * 4 +
+           1024;
+}
+
+// Most ring stages (<= kMaxStages) that fit, or 0 when fewer than kMinStages do.
+template <int MT>
+__host__ __device__ inline int pick_stages(int64_t KB, int64_t units_per_cta_max) {
+    for (int s = Layout<MT>::kMaxStages; s >= kMinStages; --s)
+        if (smem_bytes<MT>(s, KB, units_per_cta_max) <= kMaxSmem) return s;
+    return 0;
 }
 
 // Workspace: a fixed header of kMaxCounters int32 split-K counters, then float
@@ -71,7 +124,7 @@ __host__ __device__ inline int64_t smem_bytes(int64_t KB, int64_t units_per_cta_
 // expects to be zero: every successful call leaves the whole header zeroed.
 constexpr int64_t kMaxCounters = 4096;  // n-blocks, i.e. N <= 524288 on this path
 constexpr int64_t kCounterBytes = kMaxCounters * 4;
-__host__ __device__ inline int64_t workspace_bytes(int64_t NB) {
+__host__ __device__ inline int64_t workspace_bytes(int64_t NB, int64_t MT) {
     return kCounterBytes + (NB + kMaxGrid) * MT * BNW * 4;
 }
 
@@ -98,25 +151,38 @@ __device__ __forceinline__ SplitPlan split_plan(int64_t u_begin, int64_t u_end, 
     return p;
 }
 
-__global__ void __launch_bounds__(kNumThreads, 1)
+template <int MT>
+__global__ void __launch_bounds__(Roles<MT>::kNumThreads, 1)
 gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_x, const float *__restrict__ sa,
                    const float *__restrict__ sw, __nv_bfloat16 *__restrict__ y, int M, int N,
-                   int K, int *counters, float *partials, int *status, int early_weights) {
+                   int K, int *counters, float *partials, int *status, int early_weights,
+                   int stages) {
+    using Layout = decode::Layout<MT>;
+    const int kStages = stages;
+    constexpr int kStep = Layout::kStep;
+    constexpr int kGroups = Layout::kGroups;
+    constexpr uint32_t kTmemCols = Layout::kTmemCols;
+    constexpr int kPromoWarps = Roles<MT>::kPromoWarps;
+    constexpr int kPromoThreads = Roles<MT>::kPromoThreads;
+    constexpr int kCols = Roles<MT>::kCols;
+    constexpr int kSplitWarp = Roles<MT>::kSplitWarp;
+    constexpr int kNumThreads = Roles<MT>::kNumThreads;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Layout::kBarOff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Layout::bar_off(kStages));
     uint64_t *empty = full + kStages;
     uint64_t *tfull = empty + kStages;
-    uint64_t *tempty = tfull + kTmemBufs;
-    uint64_t *drain = tempty + kTmemBufs;
+    uint64_t *tempty = tfull + kGroups;
+    uint64_t *drain = tempty + kGroups;
     uint64_t *flushed = drain + 1;  // [2]: promotion -> split-K warp, one per split n-block
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Layout::kMiscOff);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Layout::kMiscOff + 4);
-    float *sa_s = reinterpret_cast<float *>(smem + Layout::kScaleOff);  // [MT][KB]
+    uint8_t *misc = smem + Layout::misc_off(kStages);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 4);
+    float *sa_s = reinterpret_cast<float *>(smem + Layout::scale_off(kStages));  // [KB][kSaRow]
     // n-blocks this CTA must reduce (it was their last contributor), or -1
-    volatile int *reduce_nb = reinterpret_cast<volatile int *>(smem + Layout::kMiscOff + 8);
+    volatile int *reduce_nb = reinterpret_cast<volatile int *>(misc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = K / BK, NB = N / BNW;
@@ -124,7 +190,9 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     const int64_t G = gridDim.x;
     const int64_t u_begin = blockIdx.x * U / G;
     const int64_t u_end = (blockIdx.x + 1) * U / G;
-    float *sw_s = sa_s + MT * KB;  // sw[u] for u in [u_begin, u_end): sw is [NB, KB] row-major
+    const int64_t n_steps = (u_end - u_begin + kStep - 1) / kStep;
+    constexpr int kSaRow = Layout::kSaRow;
+    float *sw_s = sa_s + kSaRow * KB;  // sw[u] for u in [u_begin, u_end): sw is [NB, KB] row-major
 
     allow_dependent_launch();
     if (threadIdx.x == 0) {
@@ -132,13 +200,13 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < kTmemBufs; ++b) {
+        for (int b = 0; b < kGroups; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], kPromoWarps);
         }
         mbar_init(drain, 1);
-        mbar_init(&flushed[0], 4);
-        mbar_init(&flushed[1], 4);
+        mbar_init(&flushed[0], kPromoWarps);
+        mbar_init(&flushed[1], kPromoWarps);
         *abort_flag = 0;
         reduce_nb[0] = -1;
         reduce_nb[1] = -1;
@@ -160,35 +228,50 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     // quantizer, which writes activation codes and scales only and lets this
     // kernel start after its own dependency wait.  Every other global access
     // happens after the previous kernel has completed.
+    // Units of step i: [u_begin + kStep i, min(u_end, u_begin + kStep (i + 1))).
+    auto step_units = [&](int64_t i) {
+        const int64_t left = u_end - (u_begin + kStep * i);
+        return static_cast<int>(left < kStep ? left : kStep);
+    };
     int64_t n_early = 0;
     if (early_weights && warp == 0 && lane == 0) {
         const uint64_t evict_first = l2_policy_evict_first();
-        for (int64_t u = u_begin; u < u_end && n_early < kStages; ++u, ++n_early) {
-            const int nb = static_cast<int>(u / KB), kb = static_cast<int>(u % KB);
-            mbar_arrive_expect_tx(&full[n_early], Layout::kStage);
-            tma_load_2d_hint(smem + n_early * Layout::kStage, &tmap_w, &full[n_early], kb * BK,
-                             nb * BNW, evict_first);
+        for (; n_early < n_steps && n_early < kStages; ++n_early) {
+            const int cnt = step_units(n_early);
+            mbar_arrive_expect_tx(&full[n_early], cnt * Layout::kUnit);
+            for (int j = 0; j < cnt; ++j) {
+                const int64_t u = u_begin + kStep * n_early + j;
+                tma_load_2d_hint(smem + n_early * Layout::kStage + j * Layout::kUnit, &tmap_w,
+                                 &full[n_early], static_cast<int>(u % KB) * BK,
+                                 static_cast<int>(u / KB) * BNW, evict_first);
+            }
         }
     }
     grid_dependency_wait();
 
     if (warp == 0) {
         if (lane == 0) {
-            // activation tiles of the stages whose weight blocks went out early
+            // activation tiles of the steps whose weight blocks went out early
             for (int64_t i = 0; i < n_early; ++i)
-                tma_load_2d(smem + i * Layout::kStage + Layout::kW, &tmap_x, &full[i],
-                            static_cast<int>((u_begin + i) % KB) * BK, 0);
+                for (int j = 0; j < step_units(i); ++j)
+                    tma_load_2d(smem + i * Layout::kStage + j * Layout::kUnit + Layout::kW, &tmap_x,
+                                &full[i], static_cast<int>((u_begin + kStep * i + j) % KB) * BK, 0);
             const uint64_t evict_first = l2_policy_evict_first();
             uint32_t stage = static_cast<uint32_t>(n_early % kStages);
             uint32_t phase = n_early == kStages ? 1u : 0u;
             int64_t issued = n_early;
-            for (int64_t u = u_begin + n_early; u < u_end; ++u) {
-                const int nb = static_cast<int>(u / KB), kb = static_cast<int>(u % KB);
+            for (int64_t i = n_early; i < n_steps; ++i) {
                 if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) break;
+                const int cnt = step_units(i);
                 uint8_t *st = smem + stage * Layout::kStage;
-                mbar_arrive_expect_tx(&full[stage], Layout::kStage);
-                tma_load_2d_hint(st, &tmap_w, &full[stage], kb * BK, nb * BNW, evict_first);
-                tma_load_2d(st + Layout::kW, &tmap_x, &full[stage], kb * BK, 0);
+                mbar_arrive_expect_tx(&full[stage], cnt * Layout::kUnit);
+                for (int j = 0; j < cnt; ++j) {
+                    const int64_t u = u_begin + kStep * i + j;
+                    const int nb = static_cast<int>(u / KB), kb = static_cast<int>(u % KB);
+                    tma_load_2d_hint(st + j * Layout::kUnit, &tmap_w, &full[stage], kb * BK, nb * BNW,
+                                     evict_first);
+                    tma_load_2d(st + j * Layout::kUnit + Layout::kW, &tmap_x, &full[stage], kb * BK, 0);
+                }
                 ++issued;
                 if (++stage == kStages) {
                     stage = 0;
@@ -202,116 +285,128 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = umma_idesc_e4m3(BNW, MT);
-            uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
-            for (int64_t u = u_begin; u < u_end; ++u) {
-                if (!mbar_wait(&tempty[buf], bphase ^ 1, abort_flag, status) ||
+            uint32_t stage = 0, phase = 0, grp = 0, gphase = 0;
+            for (int64_t i = 0; i < n_steps; ++i) {
+                if (!mbar_wait(&tempty[grp], gphase ^ 1, abort_flag, status) ||
                     !mbar_wait(&full[stage], phase, abort_flag, status))
                     break;
                 tc_fence_after_sync();
-                const uint32_t w_addr = smem_addr(smem + stage * Layout::kStage);
-                const uint32_t x_addr = w_addr + Layout::kW;
-                const uint32_t d_tmem = tmem_base + buf * MT;
+                const int cnt = step_units(i);
+                for (int j = 0; j < cnt; ++j) {
+                    const uint32_t w_addr = smem_addr(smem + stage * Layout::kStage + j * Layout::kUnit);
+                    const uint32_t x_addr = w_addr + Layout::kW;
+                    const uint32_t d_tmem = tmem_base + (grp * kStep + j) * MT;
 #pragma unroll
-                for (int j = 0; j < BK / 32; ++j)
-                    umma_e4m3(d_tmem, umma_desc_sw128(w_addr + 32 * j),
-                              umma_desc_sw128(x_addr + 32 * j), idesc, j > 0 ? 1u : 0u);
+                    for (int k = 0; k < BK / 32; ++k)
+                        umma_e4m3(d_tmem, umma_desc_sw128(w_addr + 32 * k),
+                                  umma_desc_sw128(x_addr + 32 * k), idesc, k > 0 ? 1u : 0u);
+                }
                 umma_commit(&empty[stage]);
-                umma_commit(&tfull[buf]);
+                umma_commit(&tfull[grp]);
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1;
                 }
-                if (++buf == kTmemBufs) {
-                    buf = 0;
-                    bphase ^= 1;
+                if (++grp == kGroups) {
+                    grp = 0;
+                    gphase ^= 1;
                 }
             }
             umma_commit(drain);
             mbar_wait(drain, 0, nullptr, status);
         }
     } else if (warp < kSplitWarp) {
-        const int quarter = warp & 3;
-        const int n_local = quarter * 32 + lane;  // weight row within the block = TMEM lane
-        const int ptid = threadIdx.x - 64;        // 0..127 among the promotion threads
-        // Stage the scales once: every activation scale (M <= 16 rows) and the
-        // weight scales of this CTA's units, so the per-unit promotion reads
-        // shared memory only.  Loads are issued in batches so their latencies
-        // overlap.
-        constexpr int kBatch = 8;
-        const int sa_total = MT * KB, sa_valid = M * KB;
-        for (int base = ptid; base < sa_total; base += 128 * kBatch) {
-            float v[kBatch];
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const int i = base + 128 * j;
-                v[j] = (i < sa_valid) ? __ldg(sa + i) : 0.0f;
-            }
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const int i = base + 128 * j;
-                if (i < sa_total) sa_s[i] = v[j];
+        const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
+        const int col0 = ((warp - 2) >> 2) * kCols;   // first token column of this thread
+        const int n_local = quarter * 32 + lane;      // weight row within the block = TMEM lane
+        const int ptid = threadIdx.x - 64;            // 0 .. kPromoThreads-1
+        // Stage the scales once: every activation scale (rows past M as 0,
+        // transposed to [KB][kSaRow]) and the weight scales of this CTA's
+        // units, so the per-unit promotion reads shared memory only.  4-byte
+        // async copies keep all of them in flight at once.  A warp copies a
+        // tile of 8 k-blocks x 4 tokens: four 32-byte global segments, and 32
+        // distinct shared-memory banks since kSaRow is 4 times an odd number.
+        const int kb_tiles = (KB + 7) / 8;
+        for (int t = ptid >> 5; t < kb_tiles * (MT / 4); t += kPromoWarps) {
+            const int kb = (t % kb_tiles) * 8 + (lane & 7);
+            const int m = (t / kb_tiles) * 4 + (lane >> 3);
+            if (kb < KB) {
+                float *dst = sa_s + kb * kSaRow + m;
+                if (m < M)
+                    cp_async_4(dst, sa + static_cast<int64_t>(m) * KB + kb);
+                else
+                    *dst = 0.0f;
             }
         }
         const int n_units = static_cast<int>(u_end - u_begin);
-        for (int base = ptid; base < n_units; base += 128 * kBatch) {
-            float v[kBatch];
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const int i = base + 128 * j;
-                v[j] = (i < n_units) ? __ldg(sw + u_begin + i) : 0.0f;
-            }
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const int i = base + 128 * j;
-                if (i < n_units) sw_s[i] = v[j];
-            }
-        }
-        named_barrier(1, 128);
+        for (int i = ptid; i < n_units; i += kPromoThreads) cp_async_4(sw_s + i, sw + u_begin + i);
+        cp_async_wait_all();
+        named_barrier(1, kPromoThreads);
 
-        uint32_t buf = 0, bphase = 0;
-        float acc[MT];
+        uint32_t grp = 0, gphase = 0;
+        float acc[kCols];
 #pragma unroll
-        for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+        for (int m = 0; m < kCols; ++m) acc[m] = 0.0f;
         int seg_kb0 = static_cast<int>(u_begin % KB);
         int split_idx = 0;
         for (int64_t u = u_begin; u < u_end; ++u) {
             const int nb = static_cast<int>(u / KB), kb = static_cast<int>(u % KB);
             const float swv = sw_s[u - u_begin];
-            float s[MT];
-#pragma unroll
-            for (int m = 0; m < MT; ++m) s[m] = sa_s[m * KB + kb] * swv;
-            if (!mbar_wait(&tfull[buf], bphase, abort_flag, status)) break;
-            tc_fence_after_sync();
-            float v[MT];
-            tmem_load16(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * MT, v);
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
-            if (++buf == kTmemBufs) {
-                buf = 0;
-                bphase ^= 1;
+            const int j = static_cast<int>((u - u_begin) % kStep);  // unit within its step
+            const bool last_of_step = j == kStep - 1 || u == u_end - 1;
+            if (j == 0) {
+                if (!mbar_wait(&tfull[grp], gphase, abort_flag, status)) break;
+                tc_fence_after_sync();
             }
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   (grp * kStep + j) * MT + col0;
+            float v[kCols];
+            if constexpr (kCols == 16)
+                tmem_load16(taddr, v);
+            else if constexpr (kCols == 32)
+                tmem_load32(taddr, v);
+            else
+                tmem_load64(taddr, v);
+            if (last_of_step) {
+                // all of this thread's TMEM columns of the step are in registers
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[grp]);
+                if (++grp == kGroups) {
+                    grp = 0;
+                    gphase ^= 1;
+                }
+            }
+            const float4 *sa4 = reinterpret_cast<const float4 *>(sa_s + kb * kSaRow + col0);
 #pragma unroll
-            for (int m = 0; m < MT; ++m) acc[m] = fmaf(v[m], s[m], acc[m]);
+            for (int i = 0; i < kCols / 4; ++i) {
+                const float4 a = sa4[i];
+                acc[4 * i + 0] = fmaf(v[4 * i + 0], a.x * swv, acc[4 * i + 0]);
+                acc[4 * i + 1] = fmaf(v[4 * i + 1], a.y * swv, acc[4 * i + 1]);
+                acc[4 * i + 2] = fmaf(v[4 * i + 2], a.z * swv, acc[4 * i + 2]);
+                acc[4 * i + 3] = fmaf(v[4 * i + 3], a.w * swv, acc[4 * i + 3]);
+            }
 
             if (kb == KB - 1 || u == u_end - 1) {
                 // end of this CTA's segment of n-block nb
                 const int col = nb * BNW + n_local;
                 if (seg_kb0 == 0 && kb == KB - 1) {
 #pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        if (m < M) y[static_cast<int64_t>(m) * N + col] = __float2bfloat16_rn(acc[m]);
+                    for (int m = 0; m < kCols; ++m)
+                        if (col0 + m < M)
+                            y[static_cast<int64_t>(col0 + m) * N + col] = __float2bfloat16_rn(acc[m]);
                 } else {
                     // hand the partial to the split-K warp
                     float *slot = partials + (static_cast<int64_t>(nb) + blockIdx.x) * (MT * BNW);
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) __stcg(slot + m * BNW + n_local, acc[m]);
+                    for (int m = 0; m < kCols; ++m)
+                        __stcg(slot + (col0 + m) * BNW + n_local, acc[m]);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&flushed[split_idx]);
                     ++split_idx;
                 }
 #pragma unroll
-                for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+                for (int m = 0; m < kCols; ++m) acc[m] = 0.0f;
                 seg_kb0 = 0;
             }
         }
@@ -340,8 +435,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
 
     // ---------------------------------------------------------------- split-K reduction
     // Every thread of the CTA joins; partial sums are added in increasing
-    // contributor order (deterministic) with the loads of up to four
-    // contributors in flight at once.
+    // contributor order (deterministic).  A thread takes kItems float4 columns
+    // at once and up to four contributors of each, so 32 loads are in flight.
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -353,30 +448,45 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         const float4 *base = reinterpret_cast<const float4 *>(
             partials + static_cast<int64_t>(nb) * (MT * BNW));
         constexpr int kSlot4 = MT * BNW / 4;  // float4s per partial slot
-        for (int item = threadIdx.x; item < M * (BNW / 4); item += kNumThreads) {
-            const int m = item / (BNW / 4), c4 = item % (BNW / 4);
-            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        constexpr int kItems = 8;
+        const int items = M * (BNW / 4);
+        for (int item0 = threadIdx.x; item0 < items; item0 += kItems * kNumThreads) {
+            float4 sum[kItems];
+#pragma unroll
+            for (int r = 0; r < kItems; ++r) sum[r] = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int c = c_first; c <= c_last; c += 4) {
-                float4 p[4];
+                float4 p[kItems][4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    p[j] = (c + j <= c_last)
-                               ? __ldcg(base + static_cast<int64_t>(c + j) * kSlot4 + m * (BNW / 4) + c4)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int r = 0; r < kItems; ++r) {
+                    const int item = item0 + r * kNumThreads;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    sum.x += p[j].x;
-                    sum.y += p[j].y;
-                    sum.z += p[j].z;
-                    sum.w += p[j].w;
+                    for (int j = 0; j < 4; ++j)
+                        p[r][j] = (c + j <= c_last && item < items)
+                                      ? __ldcg(base + static_cast<int64_t>(c + j) * kSlot4 + item)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
+#pragma unroll
+                for (int r = 0; r < kItems; ++r)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        sum[r].x += p[r][j].x;
+                        sum[r].y += p[r][j].y;
+                        sum[r].z += p[r][j].z;
+                        sum[r].w += p[r][j].w;
+                    }
             }
-            __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z, sum.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t *>(&lo);
-            pk.y = *reinterpret_cast<uint32_t *>(&hi);
-            *reinterpret_cast<uint2 *>(y + static_cast<int64_t>(m) * N + nb * BNW + 4 * c4) = pk;
+#pragma unroll
+            for (int r = 0; r < kItems; ++r) {
+                const int item = item0 + r * kNumThreads;
+                if (item >= items) break;
+                const int m = item / (BNW / 4), c4 = item % (BNW / 4);
+                __nv_bfloat162 lo = __floats2bfloat162_rn(sum[r].x, sum[r].y);
+                __nv_bfloat162 hi = __floats2bfloat162_rn(sum[r].z, sum[r].w);
+                uint2 pk;
+                pk.x = *reinterpret_cast<uint32_t *>(&lo);
+                pk.y = *reinterpret_cast<uint32_t *>(&hi);
+                *reinterpret_cast<uint2 *>(y + static_cast<int64_t>(m) * N + nb * BNW + 4 * c4) = pk;
+            }
         }
         if (threadIdx.x == 0) atomicExch(&counters[nb], 0);
     }

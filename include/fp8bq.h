@@ -140,9 +140,10 @@ FP8BQ_API fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const
  * not permitted).  The paper has no counterpart; this is a convenience of the
  * library.  Same arguments, results and accuracy as fp8bq_gemm, minus the
  * workspace.  Its scratch is a 4 MiB array inside the library (held on every
- * GPU that loads it until the process exits), so it rejects problems whose
- * scratch would exceed that with FP8BQ_ERR_WORKSPACE: with M <= 16 that means
- * N > 32512; larger M needs no scratch.  It calls no allocator.
+ * GPU that loads it until the process exits).  Problems whose split-K scratch
+ * would exceed it are rejected with FP8BQ_ERR_WORKSPACE when M <= 16 (that
+ * is, N > 32512); for 16 < M <= 128 they run on the prefill kernel instead,
+ * which needs no scratch, and M > 128 never needs any.  It calls no allocator.
  *   - The first call on a device looks up the array's device address (a
  *     one-time set-up); make that first call before any stream capture.
  *   - All calls share the one array: calls that overlap on the GPU (other

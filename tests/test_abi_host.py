@@ -135,6 +135,11 @@ def test_workspace_sizes(L):
     assert d > 0 and d % 256 == 0
     # decode split-K: counters + (N/128 + 256) slots of 16 x 128 FP32 partials
     assert d >= (72 + 256) * 16 * 128 * 4
+    # mid-size M uses the same path with a wider token tile (32, 64 or 128 rows)
+    assert g(17, 9216, 7168) == 16384 + (72 + 256) * 32 * 128 * 4
+    assert g(64, 9216, 7168) == 16384 + (72 + 256) * 64 * 128 * 4
+    assert g(65, 9216, 7168) == g(128, 9216, 7168) == 16384 + (72 + 256) * 128 * 128 * 4
+    assert g(129, 9216, 7168) == 0
     # linear adds the activation codes and scales
     assert lin(8192, 9216, 7168) >= 8192 * 7168 + 8192 * 56 * 4
     assert lin(16, 9216, 7168) >= d + 16 * 7168 + 16 * 56 * 4

@@ -5,7 +5,8 @@ The GEMM is fed the oracle's codes and scales; its BF16 output must satisfy
 dequantized operands (tolerance of the library's accuracy contract; the page
 "ProCreations/Nanbeige4.3-33B-FP8", "Compatibility and limitations", claims no
 bit-exact equivalence across kernel geometry).  Shapes span several tiles with
-ragged M tails on both the decode (M <= 16) and prefill paths; the full
+ragged M tails on the decode path (every token tile: M <= 16, 32, 64, 128)
+and the prefill path (M > 128); the full
 workload shapes are checked on sampled rows.  In the exact-arithmetic regime
 (small-integer codes, power-of-two scales) every partial sum is exact in FP32,
 so the output must equal the BF16 rounding of the exact result bit for bit.
@@ -68,7 +69,21 @@ def test_gemm_decode_path(M, N, K):
     check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
 
 
-PREFILL_SHAPES = [(17, 128, 128), (128, 256, 256), (129, 384, 1024), (255, 1152, 512),
+# one or more shapes per token tile (17..32, 33..64, 65..128), with ragged M,
+# several n-blocks split across CTAs and a K long enough that the staged scales
+# cut the ring to four stages at M > 64
+MIDM_SHAPES = [(17, 128, 128), (32, 256, 384), (33, 1024, 7168), (64, 384, 1024),
+               (65, 2048, 896), (100, 1152, 7168), (128, 256, 256), (128, 512, 21504)]
+
+
+@pytest.mark.parametrize("M,N,K", MIDM_SHAPES)
+def test_gemm_mid_m_decode_path(M, N, K):
+    _, qa, sa, qw, sw = operands(M, N, K, 300 + M)
+    y = run_gemm(qa, sa, qw, sw)
+    check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
+
+
+PREFILL_SHAPES = [(129, 384, 1024), (255, 1152, 512),
                   (1000, 512, 896), (300, 128, 7168), (2048, 2048, 384)]
 
 
@@ -84,21 +99,23 @@ def sample_rows(M, step, extra=()):
     return np.array(sorted(rows), dtype=np.int64)
 
 
-@pytest.mark.parametrize("name", ["k_proj", "qkv_m8", "o_proj_m4", "qkv_prefill", "fc",
-                                  "gate_up", "down", "o_proj_long"])
+@pytest.mark.parametrize("name", ["k_proj", "qkv_m8", "o_proj_m4", "qkv_m32", "o_proj_m128",
+                                  "qkv_m128", "qkv_prefill", "fc", "gate_up", "down",
+                                  "o_proj_long"])
 def test_gemm_full_workloads_sampled(name):
     g = workloads.by_name(name)
     x = g.make_x()
     qa, sa = oracle.quantize_act(x)
     qw, sw = oracle.quantize_weight(g.make_w())
     y = run_gemm(qa, sa, qw, sw)
-    step = 1 if g.M <= 16 else max(1, g.M // 48)
+    step = 1 if g.M <= 128 else max(1, g.M // 48)
     rows = sample_rows(g.M, step, extra=(127, 128, g.M - 129))
     ref = oracle.gemm_ref(qa, sa, qw, sw, rows=rows)
     check(bf16_to_f64(y)[rows], ref)
 
 
-@pytest.mark.parametrize("M,N,K", [(4, 256, 512), (300, 384, 640)])
+@pytest.mark.parametrize("M,N,K", [(4, 256, 512), (40, 640, 1024), (128, 384, 2048),
+                                   (300, 384, 640)])
 def test_gemm_exact_arithmetic_regime_bit_exact(M, N, K):
     rng = np.random.default_rng(M)
     small = np.array([0x00, 0x38, 0x40, 0x44, 0x48, 0xB8, 0xC0, 0xC4], np.uint8)  # 0,+-1,+-2,+-3,4
@@ -123,7 +140,7 @@ def test_gemm_identity_weight_closed_form():
     check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
 
 
-@pytest.mark.parametrize("M", [8, 600])
+@pytest.mark.parametrize("M", [8, 96, 600])
 def test_gemm_deterministic(M):
     _, qa, sa, qw, sw = operands(M, 1024, 7168, 7)
     y1 = run_gemm(qa, sa, qw, sw).cpu()
@@ -143,7 +160,7 @@ def test_gemm_empty_m_is_noop():
 # ------------------------------------------------------------------ fused linear
 
 @pytest.mark.parametrize("M,N,K", [(1, 1024, 7168), (16, 1024, 7168), (5, 384, 640),
-                                   (33, 256, 1024), (700, 384, 7168)])
+                                   (33, 256, 1024), (128, 1152, 7168), (700, 384, 7168)])
 def test_linear_matches_oracle_and_unfused_path(M, N, K):
     x, qa, sa, qw, sw = operands(M, N, K, 300 + M)
     xd = x.cuda()
@@ -182,12 +199,13 @@ def test_linear_prefill_qkv_sampled():
 
 def test_gemm_workspace_reused_across_calls():
     # split-K counters must be back at zero after every call for the next one to be right
-    shapes = [(8, 9216, 7168), (16, 1024, 7168), (3, 16384, 256), (8, 9216, 7168)]
+    shapes = [(8, 9216, 7168), (100, 1152, 7168), (3, 16384, 256), (8, 9216, 7168),
+              (64, 2048, 1024)]
     ws = torch.zeros(max(fp8bq.workspace_size(fp8bq.OP_GEMM, *s) for s in shapes),
                      dtype=torch.uint8, device="cuda")
     outs = []
     for i, (M, N, K) in enumerate(shapes):
-        _, qa, sa, qw, sw = operands(M, N, K, 40 + (i % 3))
+        _, qa, sa, qw, sw = operands(M, N, K, 40 + (i % 3) + M)
         y = fp8bq.gemm(to_dev_codes(qa), to_dev_f32(sa), to_dev_codes(qw), to_dev_f32(sw),
                        workspace=ws)
         torch.cuda.synchronize()

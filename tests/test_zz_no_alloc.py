@@ -50,7 +50,8 @@ def _noalloc_via_c_abi(qa, sa, qw, sw, y):
 
 
 @pytest.mark.parametrize("first,second", [((8, 9216, 7168), (16, 1024, 7168)),
-                                          ((1, 2048, 1024), (300, 384, 1024))])
+                                          ((1, 2048, 1024), (300, 384, 1024)),
+                                          ((100, 1152, 7168), (4, 7168, 7168))])
 def test_noalloc_matches_gemm_on_two_calls_in_a_row(first, second):
     for (M, N, K), seed in ((first, 11), (second, 12)):
         qa, sa, qw, sw = _operands(M, N, K, seed)

@@ -147,7 +147,16 @@ DRAFTER_MLP = (DRAFTER_FC, DRAFTER_GATE_UP, DRAFTER_DOWN)
 LONG_O_PROJ = Gemm("o_proj_long", 32768, HIDDEN, HIDDEN, 5, x_kind="t3",
                    t3_channels=HIDDEN // 100)
 
-ALL = (KPROJ_M16,) + DECODE_SET + (PREFILL_QKV,) + DRAFTER_MLP + (LONG_O_PROJ,)
+# workload 6: mid-size batches between the decode and prefill regimes (the
+# 128-stream aggregate decode step and a 32-row batch), fused QKV and o_proj
+MIDM_SET = tuple(
+    Gemm(f"{nm}_m{m}", m, n, HIDDEN, 6, outliers=OUTLIERS_0P1, x_seed_t=10 * i + 2 * j,
+         w_seed_t=1 + 2 * j)
+    for i, m in enumerate((32, 128))
+    for j, (nm, n) in enumerate((("qkv", QKV), ("o_proj", HIDDEN)))
+)
+
+ALL = (KPROJ_M16,) + DECODE_SET + (PREFILL_QKV,) + DRAFTER_MLP + (LONG_O_PROJ,) + MIDM_SET
 
 
 def by_name(name: str) -> Gemm:
