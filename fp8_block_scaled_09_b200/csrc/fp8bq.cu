@@ -5,8 +5,10 @@
 // single per-device symbol.  Dispatch:
 //   quantize_act     -> quantize_act_kernel (HBM-bound, persistent, bulk-copy ring)
 //   quantize_weight  -> quantize_weight_kernel (one CTA per 128x128 block)
-//   gemm, M <= 128   -> decode::gemm_decode_kernel<MT> (stream-K over weight
-//                       blocks; token tile MT = 16, 32, 64 or 128)
+//   gemm, M <= 128   -> decode::gemm_decode_kernel<MT> (token tile MT = 16, 32,
+//                       64 or 128; each n-block split over a cluster of CTAs
+//                       reduced in shared memory, or stream-K over all weight
+//                       blocks with a global split-K reduction)
 //   gemm, M > 128    -> prefill::gemm_prefill_kernel<256> (persistent tcgen05;
 //                       the CTA-pair kernel prefill2 is built but not dispatched)
 //   linear           -> quantize_act into the workspace, then the gemm path; the
@@ -64,6 +66,9 @@ std::atomic<uint64_t> g_launches{0};
 struct DeviceInfo {
     int sm_count = 0;
     int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair prefill kernel
+    // co-resident decode clusters of each size 2..8 (one CTA per SM at full
+    // shared memory); the decode plan only uses sizes whose clusters all fit
+    int cluster_capacity[9] = {};
     int *status = nullptr;  // device address of g_status
     bool supported = false;
 };
@@ -157,6 +162,26 @@ const DeviceInfo *device_info() {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode::kMaxSmem) != cudaSuccess)
             return;
+        // How many clusters of decode CTAs (one per SM at full shared memory)
+        // the GPU can hold at once, per cluster size.
+        for (int c = 2; c <= 8; ++c) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(static_cast<unsigned>(c));
+            cfg.blockDim = dim3(decode::Roles<128>::kNumThreads);
+            cfg.dynamicSmemBytes = decode::kMaxSmem;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = static_cast<unsigned>(c);
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, decode::gemm_decode_kernel<128>, &cfg) != cudaSuccess)
+                n = 0;
+            cudaGetLastError();  // clear a failed query
+            d.cluster_capacity[c] = n;
+        }
         if (cudaDeviceSynchronize() != cudaSuccess) return;
         d.supported = true;
     });
@@ -251,18 +276,65 @@ int64_t decode_grid(int64_t units, int64_t sms) {
     return std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(sms, decode::kMaxGrid), by_work));
 }
 
-// Ring stages of the decode kernel for this shape, or 0 if it does not apply.
-int decode_stages(int64_t M, int64_t N, int64_t K, int64_t sms) {
-    if (M > kDecodeMaxM || N / 128 > decode::kMaxCounters) return 0;
-    const int64_t units = (N / 128) * (K / 128);
-    const int64_t grid = decode_grid(units, sms);
-    const int64_t upc = (units + grid - 1) / grid, KB = K / 128;
-    switch (decode::token_tile(M)) {
-        case 16: return decode::pick_stages<16>(KB, upc);
-        case 32: return decode::pick_stages<32>(KB, upc);
-        case 64: return decode::pick_stages<64>(KB, upc);
-        default: return decode::pick_stages<128>(KB, upc);
+// How the decode kernel runs one shape: grid, ring stages (0: the decode
+// kernel does not apply) and cluster size (0: stream-K over the whole grid;
+// S >= 1: n-block nb on CTAs [nb S, nb S + S), one cluster of S when S >= 2).
+struct DecodePlan {
+    int64_t grid = 0;
+    int stages = 0;
+    int cluster_s = 0;
+};
+
+template <int MT>
+int pick_stages_for(int64_t KB, int64_t upc) {
+    return decode::pick_stages<MT>(KB, upc);
+}
+
+int pick_stages_mt(int MT, int64_t KB, int64_t upc) {
+    switch (MT) {
+        case 16: return pick_stages_for<16>(KB, upc);
+        case 32: return pick_stages_for<32>(KB, upc);
+        case 64: return pick_stages_for<64>(KB, upc);
+        default: return pick_stages_for<128>(KB, upc);
     }
+}
+
+// Chooses between the two modes with a cost model fitted to globaltimer traces
+// of this kernel: a unit (one 16 KB weight block) takes ~0.35 us per CTA
+// (~0.5 us with a 128-row token tile); stream-K adds ~4.4 us (~6 us) of tail
+// for its global split-K reduction, the cluster mode ~1 us (0.3 us when each
+// CTA owns a whole n-block).
+DecodePlan decode_plan(const DeviceInfo &d, int64_t M, int64_t N, int64_t K) {
+    DecodePlan p;
+    if (M > kDecodeMaxM || N / 128 > decode::kMaxCounters) return p;
+    const int64_t NB = N / 128, KB = K / 128, U = NB * KB, sms = d.sm_count;
+    const int MT = decode::token_tile(M);
+    const double t_unit = MT == 128 ? 0.5 : 0.35, tail_sk = MT == 128 ? 6.0 : 4.4;
+    const int64_t g_sk = decode_grid(U, sms);
+    const int64_t upc_sk = (U + g_sk - 1) / g_sk;
+    const double cost_sk = upc_sk * t_unit + tail_sk;
+    if (NB <= sms) {
+        // largest S <= 8 whose NB clusters are all co-resident, with a unit each
+        int64_t S = std::min<int64_t>(std::min<int64_t>(8, sms / NB), KB);
+        while (S >= 2 && NB > d.cluster_capacity[S]) --S;
+        S = std::max<int64_t>(S, 1);
+        const int64_t upc_c = (KB + S - 1) / S;
+        const double cost_c = upc_c * t_unit + (S > 1 ? 1.0 : 0.3);
+        const int st_c = pick_stages_mt(MT, KB, upc_c);
+        // the cluster reduction keeps the [MT][128] FP32 partial in the ring
+        const bool ring_holds_partial =
+            st_c > 0 && static_cast<int64_t>(st_c) * decode::kStageBytes(MT) >= int64_t(MT) * 128 * 4;
+        if (ring_holds_partial && cost_c <= cost_sk) {
+            p.grid = NB * S;
+            p.stages = st_c;
+            p.cluster_s = static_cast<int>(S);
+            return p;
+        }
+    }
+    p.grid = g_sk;
+    p.stages = pick_stages_mt(MT, KB, upc_sk);
+    p.cluster_s = 0;
+    return p;
 }
 
 size_t gemm_ws_bytes(int64_t M, int64_t N) {
@@ -292,22 +364,25 @@ template <int MT>
 cudaError_t launch_decode(const DeviceInfo &d, const uint8_t *qa, const float *sa,
                           const uint8_t *qw, const float *sw, int64_t M, int64_t N, int64_t K,
                           void *y, void *ws, cudaStream_t st, fp8bq_status *err,
-                          bool early_weights, int stages) {
+                          bool early_weights, const DecodePlan &plan) {
     CUtensorMap tw, tx;
     if (!make_tmap(&tw, qw, N, K, decode::BNW) || !make_tmap(&tx, qa, M, K, MT)) {
         *err = FP8BQ_ERR_CUDA;
         return cudaSuccess;
     }
-    const int64_t units = (N / 128) * (K / 128);
-    const int64_t grid = decode_grid(units, d.sm_count);
+    const int64_t KB = K / 128, units = (N / 128) * KB;
+    const int64_t upc = plan.cluster_s > 0 ? (KB + plan.cluster_s - 1) / plan.cluster_s
+                                           : (units + plan.grid - 1) / plan.grid;
     int *counters = static_cast<int *>(ws);
-    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes);
-    const int64_t smem = decode::smem_bytes<MT>(stages, K / 128, (units + grid - 1) / grid);
-    return launch(decode::gemm_decode_kernel<MT>, dim3(static_cast<unsigned>(grid)),
-                  dim3(decode::Roles<MT>::kNumThreads), static_cast<size_t>(smem), st, tw, tx, sa, sw,
-                  static_cast<__nv_bfloat16 *>(y), static_cast<int>(M), static_cast<int>(N),
-                  static_cast<int>(K), counters, partials, d.status, early_weights ? 1 : 0,
-                  stages);
+    float *partials =
+        ws ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes) : nullptr;
+    const int64_t smem = decode::smem_bytes<MT>(plan.stages, KB, upc);
+    return launch_clustered(decode::gemm_decode_kernel<MT>, dim3(static_cast<unsigned>(plan.grid)),
+                            dim3(decode::Roles<MT>::kNumThreads), static_cast<size_t>(smem), st,
+                            plan.cluster_s > 1 ? static_cast<unsigned>(plan.cluster_s) : 1u, tw, tx,
+                            sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
+                            static_cast<int>(N), static_cast<int>(K), counters, partials, d.status,
+                            early_weights ? 1 : 0, plan.stages, plan.cluster_s);
 }
 
 // early_weights: the decode kernel may request its first weight blocks before
@@ -318,16 +393,17 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
                         void *y, void *ws, cudaStream_t st, fp8bq_status *err,
                         bool early_weights = false, bool allow_decode = true) {
     *err = FP8BQ_OK;
-    if (const int stages = allow_decode ? decode_stages(M, N, K, d.sm_count) : 0) {
+    const DecodePlan plan = decode_plan(d, M, N, K);
+    if (plan.stages > 0 && (allow_decode || plan.cluster_s > 0)) {
         switch (decode::token_tile(M)) {
             case 16:
-                return launch_decode<16>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, stages);
+                return launch_decode<16>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, plan);
             case 32:
-                return launch_decode<32>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, stages);
+                return launch_decode<32>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, plan);
             case 64:
-                return launch_decode<64>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, stages);
+                return launch_decode<64>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, plan);
             default:
-                return launch_decode<128>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, stages);
+                return launch_decode<128>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, plan);
         }
     } else if (kUsePairPrefill && d.pair_clusters > 0 && M > prefill::BM) {
         // CTA pairs: each CTA loads 128 rows of A and 128 of the 256 weight rows

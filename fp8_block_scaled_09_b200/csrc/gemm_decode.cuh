@@ -27,7 +27,16 @@
 //               counter increment), so promotion never waits on either; if the
 //               CTA was an n-block's last contributor, all warps reduce it after
 //               the main loop.
-// Stream-K: units u = nb * KB + kb are split into gridDim.x contiguous ranges.
+// Two ways to spread the units over CTAs, chosen per launch:
+// Cluster split (cluster_s >= 1, when N/128 <= the SM count): CTA c works on
+// n-block c / S, k-blocks [r KB / S, (r+1) KB / S) with r = c mod S, and the S
+// CTAs of an n-block form a thread-block cluster.  At the end each stores its
+// partial in its own shared memory; after a cluster barrier CTA r sums slice r
+// of the n-block's output over the S partials (in rank order, read through
+// distributed shared memory), writes it in BF16, and a second barrier keeps the
+// partials alive until every peer has read them.  No global workspace is used.
+// Stream-K (cluster_s == 0): units u = nb * KB + kb are split into gridDim.x
+// contiguous ranges.
 // An n-block whose K range lies inside one CTA is written straight to Y in
 // BF16.  Otherwise each contributing CTA c stores its FP32 partial in slot
 // nb + c of the workspace and increments counter[nb]; the last to arrive sums
@@ -110,6 +119,11 @@ __host__ __device__ inline int64_t smem_bytes(int stages, int64_t KB, int64_t un
            1024;
 }
 
+// Bytes of one ring slot for a token tile.
+__host__ __device__ constexpr int64_t kStageBytes(int MT) {
+    return step_units_of(MT) * (int64_t(BNW) * BK + int64_t(MT) * BK);
+}
+
 // Most ring stages (<= kMaxStages) that fit, or 0 when fewer than kMinStages do.
 template <int MT>
 __host__ __device__ inline int pick_stages(int64_t KB, int64_t units_per_cta_max) {
@@ -157,7 +171,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_x, const float *__restrict__ sa,
                    const float *__restrict__ sw, __nv_bfloat16 *__restrict__ y, int M, int N,
                    int K, int *counters, float *partials, int *status, int early_weights,
-                   int stages) {
+                   int stages, int cluster_s) {
     using Layout = decode::Layout<MT>;
     const int kStages = stages;
     constexpr int kStep = Layout::kStep;
@@ -188,8 +202,15 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     const int KB = K / BK, NB = N / BNW;
     const int64_t U = static_cast<int64_t>(NB) * KB;
     const int64_t G = gridDim.x;
-    const int64_t u_begin = blockIdx.x * U / G;
-    const int64_t u_end = (blockIdx.x + 1) * U / G;
+    int64_t u_begin, u_end;
+    if (cluster_s > 0) {
+        const int64_t nb = blockIdx.x / cluster_s, r = blockIdx.x % cluster_s;
+        u_begin = nb * KB + r * KB / cluster_s;
+        u_end = nb * KB + (r + 1) * KB / cluster_s;
+    } else {
+        u_begin = blockIdx.x * U / G;
+        u_end = (blockIdx.x + 1) * U / G;
+    }
     const int64_t n_steps = (u_end - u_begin + kStep - 1) / kStep;
     constexpr int kSaRow = Layout::kSaRow;
     float *sw_s = sa_s + kSaRow * KB;  // sw[u] for u in [u_begin, u_end): sw is [NB, KB] row-major
@@ -395,6 +416,13 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                     for (int m = 0; m < kCols; ++m)
                         if (col0 + m < M)
                             y[static_cast<int64_t>(col0 + m) * N + col] = __float2bfloat16_rn(acc[m]);
+                } else if (cluster_s > 0) {
+                    // the CTA's whole range is this one segment, and every MMA
+                    // that read the ring has completed: the ring holds the
+                    // partial [MT][128] for the cluster reduction
+                    float *red = reinterpret_cast<float *>(smem);
+#pragma unroll
+                    for (int m = 0; m < kCols; ++m) red[(col0 + m) * BNW + n_local] = acc[m];
                 } else {
                     // hand the partial to the split-K warp
                     float *slot = partials + (static_cast<int64_t>(nb) + blockIdx.x) * (MT * BNW);
@@ -415,7 +443,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         // Publishes each split n-block's partial and learns whether this CTA was
         // the last contributor; the reduction itself runs after the main loop on
         // all threads of the CTA.
-        const SplitPlan plan = split_plan(u_begin, u_end, KB);
+        const SplitPlan plan = cluster_s > 0 ? SplitPlan{} : split_plan(u_begin, u_end, KB);
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             if (i >= plan.count) break;
@@ -431,6 +459,38 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 reduce_nb[i] = (atomicAdd(&counters[nb], 1) == c_last - c_first) ? nb : -1;
             }
         }
+    }
+
+    if (cluster_s > 1) {
+        // ------------------------------------------------------------ cluster reduction
+        __syncwarp();
+        cluster_sync();
+        const int S = cluster_s;
+        const int r = static_cast<int>(blockIdx.x % S);
+        const int64_t nb = blockIdx.x / S;
+        const uint32_t red = smem_addr(smem);
+        const int items = M * (BNW / 4);  // float4 columns of the n-block's output
+        const int i0 = r * items / S, i1 = (r + 1) * items / S;
+        for (int item = i0 + static_cast<int>(threadIdx.x); item < i1; item += kNumThreads) {
+            const int m = item / (BNW / 4), c4 = item % (BNW / 4);
+            const uint32_t off = static_cast<uint32_t>((m * BNW + 4 * c4) * 4);
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int p = 0; p < S; ++p) {  // rank order = K order
+                const float4 v = ld_shared_cluster_v4(map_to_cta(red + off, static_cast<uint32_t>(p)));
+                sum.x += v.x;
+                sum.y += v.y;
+                sum.z += v.z;
+                sum.w += v.w;
+            }
+            __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z, sum.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t *>(&lo);
+            pk.y = *reinterpret_cast<uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(y + static_cast<int64_t>(m) * N + nb * BNW + 4 * c4) = pk;
+        }
+        __syncwarp();
+        cluster_sync();  // peers may still be reading this CTA's partial until here
     }
 
     // ---------------------------------------------------------------- split-K reduction

@@ -57,9 +57,13 @@ def check(y, ref):
     assert ok, f"worst error / bound = {ratio:.3f} (rms(ref) = {rms:.4g})"
 
 
+# Up to 148 n-blocks the decode kernel splits each n-block over a cluster of
+# CTAs (sizes 1-8: e.g. 2 for QKV, 3 for (2, 256, 384), 5 for (7, 640, 640), 8
+# for k_proj); beyond that it runs stream-K with the global split-K reduction
+# ((4, 19200, 512), (3, 32768, 256)).
 DECODE_SHAPES = [(1, 128, 128), (1, 1024, 7168), (2, 256, 384), (4, 9216, 7168),
                  (8, 7168, 7168), (15, 384, 1024), (16, 1024, 7168), (16, 128, 21504),
-                 (3, 16384, 256)]
+                 (3, 16384, 256), (7, 640, 640), (4, 19200, 512), (3, 32768, 256)]
 
 
 @pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
@@ -73,7 +77,8 @@ def test_gemm_decode_path(M, N, K):
 # several n-blocks split across CTAs and a K long enough that the staged scales
 # cut the ring to four stages at M > 64
 MIDM_SHAPES = [(17, 128, 128), (32, 256, 384), (33, 1024, 7168), (64, 384, 1024),
-               (65, 2048, 896), (100, 1152, 7168), (128, 256, 256), (128, 512, 21504)]
+               (65, 2048, 896), (100, 1152, 7168), (128, 256, 256), (128, 512, 21504),
+               (40, 20480, 256), (128, 19200, 384)]
 
 
 @pytest.mark.parametrize("M,N,K", MIDM_SHAPES)
