@@ -70,6 +70,9 @@ def _load():
         lib.oracle_quantize_weight.argtypes = [P, I, I, P, P]
         lib.oracle_gemm_ref.argtypes = [P, P, P, P, I, I, I, P, I, P]
         lib.oracle_bf16_round.argtypes = [ctypes.c_double]
+        lib.oracle_kv_write.argtypes = [P, P, I, I, I, P, I, I, P, P]
+        lib.oracle_kv_write.restype = ctypes.c_int64
+        lib.oracle_silu_mul.argtypes = [P, I, I, P]
         lib.oracle_bf16_round.restype = ctypes.c_uint16
         _lib = lib
         return lib
@@ -177,3 +180,47 @@ def bf16_round(v: np.ndarray) -> np.ndarray:
     out = np.fromiter((lib.oracle_bf16_round(float(t)) for t in flat), dtype=np.uint16,
                       count=flat.size)
     return out.reshape(v.shape)
+
+
+def kv_write(k, v, loc, k_cache: np.ndarray, v_cache: np.ndarray) -> int:
+    """FP8 E4M3 KV-cache write with unit scales, in place on the host caches.
+
+    k, v: BF16 [T, width] (torch or numpy bit patterns; any row stride); loc:
+    int64 [T]; k_cache, v_cache: uint8 [num_slots, slot_bytes] with slot_bytes
+    >= width.  Returns the number of rows skipped for an out-of-range slot."""
+    kb, vb = _bf16_strided(k), _bf16_strided(v)
+    T, width = kb.shape[0], kb.shape[1]
+    assert vb.shape == (T, width)
+    row_stride = kb.strides[0] // 2
+    assert vb.strides[0] // 2 == row_stride and kb.strides[1] == 2 and vb.strides[1] == 2
+    loc = np.ascontiguousarray(loc, dtype=np.int64)
+    assert k_cache.dtype == np.uint8 and k_cache.flags.c_contiguous and k_cache.shape == v_cache.shape
+    num_slots, slot_bytes = k_cache.shape
+    assert slot_bytes >= width
+    # a strided row view: pass its first element's address with the row stride
+    kp = ctypes.c_void_p(kb.ctypes.data)
+    vp = ctypes.c_void_p(vb.ctypes.data)
+    return int(_load().oracle_kv_write(kp, vp, row_stride, T, width, _ptr(loc), num_slots,
+                                       slot_bytes, _ptr(k_cache), _ptr(v_cache)))
+
+
+def silu_mul(gu) -> np.ndarray:
+    """FP64 silu(gate) * up of a BF16 [M, 2I] gate/up tensor (gate first)."""
+    g = _bf16_bits(gu)
+    M, two_i = g.shape
+    h = np.empty((M, two_i // 2), dtype=np.float64)
+    _load().oracle_silu_mul(_ptr(g), M, two_i // 2, _ptr(h))
+    return h
+
+
+def _bf16_strided(x) -> np.ndarray:
+    """BF16 bit patterns as a uint16 [rows, cols] array.  A numpy uint16 array is
+    used as is (a column slice of a wider array keeps its row stride); a torch
+    BF16 tensor is copied to a contiguous host array."""
+    import torch
+    if isinstance(x, torch.Tensor):
+        assert x.dtype == torch.bfloat16 and x.dim() == 2
+        return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    a = np.asarray(x)
+    assert a.dtype == np.uint16 and a.ndim == 2 and a.strides[1] == 2
+    return a

@@ -294,3 +294,71 @@ uint16_t oracle_bf16_round(double v)
     memcpy(&u, &f, sizeof u);
     return (uint16_t)(sign | ((u >> 16) & 0x7FFF));
 }
+
+/*
+ * FP8 E4M3 KV-cache write with unit scales (page "ProCreations/Nanbeige4.3-33B-FP8",
+ * section "Serving" and the "Speed on Vega" table: --kv-cache-dtype fp8_e4m3
+ * with unit cache scales).  Each K and V element x is stored as the code of
+ * fl32(x / 1) = x under the same rule as every other code here: nearest E4M3,
+ * ties to even, saturating at 448.  The page defines no behaviour for
+ * non-finite projections; this oracle gives NaN the NaN code (0x7F, sign kept)
+ * and +-infinity the saturated code +-448.
+ *
+ * k, v      : BF16 bit patterns, row t at k + t * row_stride (elements); width
+ *             elements per row (all KV heads of the token)
+ * loc       : int64 [T], the cache slot of each row
+ * k_cache,
+ * v_cache   : E4M3 codes, slot s at k_cache + s * slot_stride (bytes)
+ * Rows whose slot is outside [0, num_slots) are not written; the count of such
+ * rows is returned.
+ */
+static uint8_t kv_code(uint16_t h)
+{
+    float x = bf16_bits_to_float(h);
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    if (isnan(x))
+        return sign | 0x7F;
+    if (isinf(x))
+        return sign | 0x7E;
+    return oracle_e4m3_encode(x / 1.0f);
+}
+
+int64_t oracle_kv_write(const uint16_t *k, const uint16_t *v, int64_t row_stride, int64_t T,
+                        int64_t width, const int64_t *loc, int64_t num_slots,
+                        int64_t slot_stride, uint8_t *k_cache, uint8_t *v_cache)
+{
+    int64_t skipped = 0;
+    for (int64_t t = 0; t < T; t++) {
+        int64_t s = loc[t];
+        if (s < 0 || s >= num_slots) {
+            skipped++;
+            continue;
+        }
+        for (int64_t i = 0; i < width; i++) {
+            k_cache[s * slot_stride + i] = kv_code(k[t * row_stride + i]);
+            v_cache[s * slot_stride + i] = kv_code(v[t * row_stride + i]);
+        }
+    }
+    return skipped;
+}
+
+/*
+ * SiLU-gated product feeding the down projection (page "ProCreations/
+ * Nanbeige4.3-33B-FP8", introduction: every linear layer, the MLP's down
+ * projection included, takes dynamically quantized activations).  The fused
+ * gate/up output gu is [M, 2I]: gate = columns [0, I), up = [I, 2I).
+ *   h[m, i] = silu(gate) * up = gate / (1 + exp(-gate)) * up, here in FP64.
+ * The quantized down-projection input is then the group-128 quantization of
+ * the BF16 rounding of h (oracle_quantize_act on those BF16 values).
+ */
+void oracle_silu_mul(const uint16_t *gu, int64_t M, int64_t I, double *h)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t i = 0; i < I; i++) {
+            double g = (double)bf16_bits_to_float(gu[m * 2 * I + i]);
+            double u = (double)bf16_bits_to_float(gu[m * 2 * I + I + i]);
+            h[m * I + i] = g / (1.0 + exp(-g)) * u;
+        }
+    }
+}
