@@ -53,7 +53,7 @@ ROTATE = 4                   # device copies of each decode weight
 # DRAM bytes (read + write) of one decode GEMM launch, o_proj M=1 (7168 x 7168), from the ncu
 # capture summarised in profiles/gemm_decode_kernel_o_proj_m1.md; scaled to other shapes by
 # their algorithmic bytes (the capture shows DRAM bytes = algorithmic bytes within 0.04%).
-DECODE_TRAFFIC_CAPTURE = {"shape": (1, 7168, 7168), "dram_bytes": 51_441_664 + 4_096,
+DECODE_TRAFFIC_CAPTURE = {"shape": (1, 7168, 7168), "dram_bytes": 51_472_640 + 28_928,
                           "source": "profiles/gemm_decode_kernel_o_proj_m1.md"}
 DECODE_WORKLOAD = ("decode GEMV set: fp8bq_linear, M in {1,4,8} x {fused QKV W[9216,7168], "
                    "o_proj W[7168,7168]}, E4M3 128x128-blocked weights, X BF16 N(0,1) with "
@@ -380,7 +380,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                 "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": traffic,
                 "traffic_source": f"ncu dram read+write of one launch ({DECODE_TRAFFIC_CAPTURE['source']}),"
                                   " scaled to this mix by algorithmic bytes",
-                "kernel": "fp8bq::decode::gemm_decode_kernel",
+                "kernel": "fp8bq::decode::gemm_decode_kernel<16> (cluster split)",
                 "avg_launch_us": gms * 1e3 / gemm_launches,
                 "algorithmic_bytes_per_launch": gemm_step_bytes / gemm_kernels_per_step,
                 "peak_source": f"{peaks['source']} HBM copy bandwidth"}
@@ -522,6 +522,51 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
         "timing": f"mean of {iters} graph replays, CUDA events, L2 flushed (256 MB write + read) before each",
     }
 
+    # FP8 KV-cache write with unit scales: K and V of the fused QKV output
+    kv_rows = []
+    for T in (2048, 32768):
+        gen = torch.Generator(device=dev).manual_seed(T)
+        qkv = torch.randn((T, 9216), generator=gen, device=dev).mul_(3).to(torch.bfloat16)
+        loc = torch.randperm(T, generator=gen, device=dev)
+        kc = torch.empty((T, 1024), dtype=torch.uint8, device=dev)
+        vc = torch.empty_like(kc)
+        kk, vv = qkv[:, 7168:8192], qkv[:, 8192:]
+        with clocks:
+            tk = flushed_ms(torch, lambda: fp8bq.kv_write_e4m3(kk, vv, loc, kc, vc), iters, warm, flush)
+        mk = statistics.fmean(tk)
+        kbytes = T * (6 * 1024 + 8)
+        kv_rows.append({"T": T, "width": 1024, "us": mk * 1e3, "gbs": kbytes / (mk * 1e-3) / 1e9,
+                        "frac_hbm": kbytes / (mk * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                        "algorithmic_bytes": kbytes})
+        del qkv, loc, kc, vc
+    out["kv_write"] = {"rows": kv_rows,
+                       "bytes": "per token: K and V read in BF16 (4 x 1024 B), written in E4M3 "
+                                "(2 x 1024 B), slot index 8 B"}
+
+    # SiLU-gated product quantized for the down projection (drafter MLP shape)
+    Mg, Ig = 4096, 8192
+    gen = torch.Generator(device=dev).manual_seed(4)
+    gu = torch.randn((Mg, 2 * Ig), generator=gen, device=dev).mul_(2).to(torch.bfloat16)
+    qh = torch.empty((Mg, Ig), dtype=torch.uint8, device=dev)
+    sh = torch.empty((Mg, Ig // 128), dtype=torch.float32, device=dev)
+    hb = torch.empty((Mg, Ig), dtype=torch.bfloat16, device=dev)
+
+    def unfused():
+        torch.mul(torch.nn.functional.silu(gu[:, :Ig]), gu[:, Ig:], out=hb)
+        fp8bq.quantize_act(hb, qh, sh)
+
+    with clocks:
+        tf = flushed_ms(torch, lambda: fp8bq.silu_mul_quantize(gu, qh, sh), iters, warm, flush)
+        tu = flushed_ms(torch, unfused, iters, warm, flush)
+    mf, mu = statistics.fmean(tf), statistics.fmean(tu)
+    sbytes = Mg * 2 * Ig * 2 + Mg * Ig + Mg * (Ig // 128) * 4
+    out["silu_mul_quantize"] = {
+        "shape": {"M": Mg, "I": Ig}, "us": mf * 1e3, "gbs": sbytes / (mf * 1e-3) / 1e9,
+        "frac_hbm": sbytes / (mf * 1e-3) / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": sbytes,
+        "unfused_us": mu * 1e3,
+        "unfused": "torch silu * up into BF16 h, then fp8bq.quantize_act(h): context only"}
+    del gu, qh, sh, hb
+
     rows = [pq]
     for g in (W.KPROJ_M16,) + W.DRAFTER_MLP + (W.LONG_O_PROJ,):
         rows.append(shape_result(g, True))
@@ -558,6 +603,18 @@ def run_profile_case(case: str) -> None:
         x = g.make_x().to(dev)
         for _ in range(3):
             fp8bq.quantize_act(x)
+    elif case == "kv":
+        T = 32768
+        qkv = torch.randn((T, 9216), device=dev).to(torch.bfloat16)
+        loc = torch.randperm(T, device=dev)
+        kc = torch.empty((T, 1024), dtype=torch.uint8, device=dev)
+        vc = torch.empty_like(kc)
+        for _ in range(3):
+            fp8bq.kv_write_e4m3(qkv[:, 7168:8192], qkv[:, 8192:], loc, kc, vc)
+    elif case == "silu":
+        gu = torch.randn((4096, 16384), device=dev).mul_(2).to(torch.bfloat16)
+        for _ in range(3):
+            fp8bq.silu_mul_quantize(gu)
     else:
         gs = {"decode": W.DECODE_SET, "midm": W.MIDM_SET}.get(case, (W.PREFILL_QKV,))
         wq = {}
@@ -587,7 +644,7 @@ def main() -> None:
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--quick", action="store_true", help="decode set only (no prefill/workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=("decode", "midm", "prefill", "quantize"),
+    ap.add_argument("--only", choices=("decode", "midm", "prefill", "quantize", "kv", "silu"),
                     help="profiling case: run one kernel family a few times, print a short line")
     args = ap.parse_args()
 

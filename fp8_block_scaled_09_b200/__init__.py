@@ -13,6 +13,8 @@ Functions (names follow the C ABI without the ``fp8bq_`` prefix):
 * ``quantize_weight(w)``     BF16 [N, K] -> (E4M3 codes uint8 [N, K], FP32 [N/128, K/128])
 * ``gemm(qa, sa, qw, sw)``   -> BF16 [M, N]
 * ``linear(x, qw, sw)``      -> BF16 [M, N], activation quantization fused into the call
+* ``kv_write_e4m3(k, v, loc, k_cache, v_cache)``  E4M3 unit-scale KV-cache write (in place)
+* ``silu_mul_quantize(gu)``  BF16 [M, 2I] gate|up -> (codes [M, I], FP32 [M, I/128])
 """
 from __future__ import annotations
 
@@ -26,6 +28,7 @@ __all__ = [
     "Fp8bqError", "lib", "quantize_act", "quantize_weight", "gemm", "gemm_noalloc", "linear",
     "workspace_size", "new_workspace", "workspace_init", "last_device_status",
     "launch_count", "status_string", "selftest_timeout", "OP_GEMM", "OP_LINEAR", "LIB_PATH",
+    "kv_write_e4m3", "silu_mul_quantize",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bq.so")
@@ -35,7 +38,7 @@ OP_LINEAR = 1
 STATUS_NAMES = {
     0: "FP8BQ_OK", 1: "FP8BQ_ERR_INVALID_ARG", 2: "FP8BQ_ERR_UNSUPPORTED_SHAPE",
     3: "FP8BQ_ERR_MISALIGNED", 4: "FP8BQ_ERR_WORKSPACE", 5: "FP8BQ_ERR_CUDA",
-    6: "FP8BQ_ERR_TIMEOUT", 7: "FP8BQ_ERR_NO_DEVICE",
+    6: "FP8BQ_ERR_TIMEOUT", 7: "FP8BQ_ERR_NO_DEVICE", 8: "FP8BQ_ERR_INDEX",
 }
 
 _lock = threading.Lock()
@@ -66,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_linear.argtypes = [P, P, P, I, I, I, P, P, S, P]
         L.fp8bq_gemm_noalloc.argtypes = [P, P, P, P, I, I, I, P, P]
         L.fp8bq_selftest_timeout.argtypes = [ctypes.c_uint32, P]
+        L.fp8bq_kv_write_e4m3.argtypes = [P, P, I, I, I, P, P, P, I, I, P]
+        L.fp8bq_silu_mul_quantize.argtypes = [P, I, I, P, P, P, P]
         L.fp8bq_workspace_size.argtypes = [ctypes.c_int, I, I, I]
         L.fp8bq_workspace_size.restype = S
         L.fp8bq_workspace_init.argtypes = [P, S, P]
@@ -78,7 +83,7 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_version.restype = ctypes.c_int
         for name in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
                      "fp8bq_workspace_init", "fp8bq_last_device_status", "fp8bq_gemm_noalloc",
-                     "fp8bq_selftest_timeout"):
+                     "fp8bq_selftest_timeout", "fp8bq_kv_write_e4m3", "fp8bq_silu_mul_quantize"):
             getattr(L, name).restype = st
         _lib = L
         return L
@@ -225,3 +230,53 @@ def selftest_timeout(limit_us: int = 20000) -> None:
 
 def launch_count() -> int:
     return int(lib().fp8bq_launch_count())
+
+
+def kv_write_e4m3(k: torch.Tensor, v: torch.Tensor, loc: torch.Tensor, k_cache: torch.Tensor,
+                  v_cache: torch.Tensor) -> None:
+    """fp8bq_kv_write_e4m3: k_cache[loc[t], :W] = e4m3(k[t]) and the same for v, with
+    unit scales.  k, v: BF16 [T, W] with unit column stride and a shared row stride (e.g.
+    column slices of the fused QKV output); loc: int64 [T]; caches: uint8 or
+    float8_e4m3fn [num_slots, slot_bytes], slot_bytes >= W.  Out-of-range slots are
+    skipped on the device and reported through last_device_status()."""
+    for t, name in ((k, "k"), (v, "v")):
+        if t.dtype != torch.bfloat16 or t.device.type != "cuda" or t.dim() != 2 or t.stride(1) != 1:
+            raise ValueError(f"{name} must be a 2-D CUDA BF16 tensor with unit column stride")
+    if k.shape != v.shape or k.stride(0) != v.stride(0):
+        raise ValueError("k and v must have the same shape and row stride")
+    k_cache, v_cache = _codes(k_cache), _codes(v_cache)
+    _need(k_cache, torch.uint8, "k_cache")
+    _need(v_cache, torch.uint8, "v_cache")
+    _need(loc, torch.int64, "loc")
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 2:
+        raise ValueError("k_cache and v_cache must be [num_slots, slot_bytes] of the same shape")
+    T, W = k.shape
+    if loc.shape != (T,):
+        raise ValueError("loc must be int64 [T]")
+    _check(lib().fp8bq_kv_write_e4m3(_ptr(k), _ptr(v), k.stride(0), T, W, _ptr(loc),
+                                     _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
+                                     k_cache.shape[1], _stream(k)), "fp8bq_kv_write_e4m3")
+
+
+def silu_mul_quantize(gu: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None,
+                      h: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """fp8bq_silu_mul_quantize: gu BF16 [M, 2I] (gate, then up) -> the group-128
+    quantization of h = BF16(silu(gate) * up): (codes uint8 [M, I], scales FP32
+    [M, I/128]).  Pass h (BF16 [M, I]) to also receive h itself."""
+    _need(gu, torch.bfloat16, "gu")
+    M, two_i = gu.shape
+    if two_i % 2:
+        raise ValueError("gu must have an even number of columns (gate | up)")
+    I = two_i // 2
+    if q is None:
+        q = torch.empty((M, I), dtype=torch.uint8, device=gu.device)
+    if s is None:
+        s = torch.empty((M, I // 128 if I % 128 == 0 else 0), dtype=torch.float32, device=gu.device)
+    q = _codes(q)
+    _need(q, torch.uint8, "q")
+    _need(s, torch.float32, "s")
+    if h is not None:
+        _need(h, torch.bfloat16, "h")
+    _check(lib().fp8bq_silu_mul_quantize(_ptr(gu), M, I, _ptr(q), _ptr(s), _ptr(h), _stream(gu)),
+           "fp8bq_silu_mul_quantize")
+    return q, s

@@ -11,6 +11,8 @@
 //                       blocks with a global split-K reduction)
 //   gemm, M > 128    -> prefill::gemm_prefill_kernel<256> (persistent tcgen05;
 //                       the CTA-pair kernel prefill2 is built but not dispatched)
+//   kv_write_e4m3    -> kv_write_e4m3_kernel (warp per K/V row, slot scatter)
+//   silu_mul_quantize-> silu_mul_quantize_kernel (half-warp per 128-channel group)
 //   linear           -> quantize_act into the workspace, then the gemm path; the
 //                       decode kernel then streams its first weight blocks while
 //                       the quantizer still runs (programmatic dependent launch)
@@ -28,7 +30,9 @@
 #include "gemm_prefill.cuh"
 #include "gemm_prefill2.cuh"
 #include "ptx.cuh"
+#include "kv_cache.cuh"
 #include "quantize.cuh"
+#include "silu_quant.cuh"
 
 namespace fp8bq {
 
@@ -484,6 +488,55 @@ fp8bq_status fp8bq_quantize_weight(const void *w_bf16, int64_t N, int64_t K, uin
                             static_cast<const uint16_t *>(w_bf16), K, q_e4m3, sw));
 }
 
+fp8bq_status fp8bq_kv_write_e4m3(const void *k_bf16, const void *v_bf16, int64_t row_stride,
+                                 int64_t T, int64_t width, const int64_t *loc, uint8_t *k_cache,
+                                 uint8_t *v_cache, int64_t num_slots, int64_t slot_stride,
+                                 void *stream) {
+    if (T < 0 || width <= 0 || row_stride < width || slot_stride < width || num_slots < 0)
+        return FP8BQ_ERR_INVALID_ARG;
+    if (width % 8 != 0 || row_stride % 8 != 0 || slot_stride % 16 != 0 || width / 8 > kMaxDim)
+        return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    if (T > 0 && row_stride > kMaxBytes / 2 / T) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    if (num_slots > 0 && slot_stride > kMaxBytes / num_slots) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return FP8BQ_OK;
+    if (!k_bf16 || !v_bf16 || !loc || !k_cache || !v_cache) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(loc) & 7u) != 0)
+        return FP8BQ_ERR_MISALIGNED;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    const int64_t blocks = std::min<int64_t>((2 * T + kKvWarps - 1) / kKvWarps,
+                                             static_cast<int64_t>(d->sm_count) * 8);
+    return from_cuda(launch(kv_write_e4m3_kernel, dim3(static_cast<unsigned>(blocks)),
+                            dim3(kKvThreads), 0, static_cast<cudaStream_t>(stream),
+                            static_cast<const uint16_t *>(k_bf16),
+                            static_cast<const uint16_t *>(v_bf16), row_stride, T,
+                            static_cast<int>(width / 8), loc, k_cache, v_cache, num_slots,
+                            slot_stride, d->status));
+}
+
+fp8bq_status fp8bq_silu_mul_quantize(const void *gu_bf16, int64_t M, int64_t I, uint8_t *q_e4m3,
+                                     float *s, void *h_bf16, void *stream) {
+    fp8bq_status st = check_mk(M, I);
+    if (st != FP8BQ_OK) return st;
+    if (M > 0 && 2 * I > kMaxBytes / 2 / M) return FP8BQ_ERR_UNSUPPORTED_SHAPE;  // gu [M, 2I]
+    if (M == 0) return FP8BQ_OK;
+    if (!gu_bf16 || !q_e4m3 || !s) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(gu_bf16) || !aligned16(q_e4m3) || !aligned16(s) ||
+        (h_bf16 != nullptr && !aligned16(h_bf16)))
+        return FP8BQ_ERR_MISALIGNED;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    const int64_t groups = M * (I / 128);
+    const int64_t warps = (groups + 1) / 2;
+    const int64_t blocks = std::min<int64_t>((warps + kSiluThreads / 32 - 1) / (kSiluThreads / 32),
+                                             static_cast<int64_t>(d->sm_count) * 16);
+    return from_cuda(launch(silu_mul_quantize_kernel, dim3(static_cast<unsigned>(blocks)),
+                            dim3(kSiluThreads), 0, static_cast<cudaStream_t>(stream),
+                            static_cast<const uint4 *>(gu_bf16), M, I,
+                            reinterpret_cast<uint2 *>(q_e4m3), s, static_cast<uint4 *>(h_bf16)));
+}
+
 size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {
     if (check_mnk(M, N, K) != FP8BQ_OK || M == 0) return 0;
     if (op == FP8BQ_OP_GEMM) return gemm_ws_bytes(M, N);
@@ -567,6 +620,7 @@ const char *fp8bq_status_string(fp8bq_status status) {
         case FP8BQ_ERR_CUDA: return "CUDA runtime or driver call failed";
         case FP8BQ_ERR_TIMEOUT: return "a kernel abandoned a bounded wait (timeout)";
         case FP8BQ_ERR_NO_DEVICE: return "no sm_100 device is current";
+        case FP8BQ_ERR_INDEX: return "a row's cache slot was out of range (the row was skipped)";
     }
     return "unknown status";
 }

@@ -72,7 +72,8 @@ typedef enum {
     FP8BQ_ERR_WORKSPACE = 4,         /* workspace missing or smaller than required */
     FP8BQ_ERR_CUDA = 5,              /* a CUDA runtime or driver call failed */
     FP8BQ_ERR_TIMEOUT = 6,           /* a kernel abandoned a bounded wait */
-    FP8BQ_ERR_NO_DEVICE = 7          /* no sm_100 device is current */
+    FP8BQ_ERR_NO_DEVICE = 7,         /* no sm_100 device is current */
+    FP8BQ_ERR_INDEX = 8              /* device side: a row's slot index was out of range */
 } fp8bq_status;
 
 /* Operation selector for fp8bq_workspace_size. */
@@ -132,6 +133,52 @@ FP8BQ_API fp8bq_status fp8bq_gemm(const uint8_t *qa, const float *sa, const uint
 FP8BQ_API fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const float *sw, int64_t M,
                           int64_t N, int64_t K, void *y_bf16, void *workspace, size_t ws_bytes,
                           void *stream);
+
+/*
+ * FP8 E4M3 KV-cache write with unit scales (page "ProCreations/Nanbeige4.3-33B-FP8",
+ * "Serving" and the "Speed on Vega" table: --kv-cache-dtype fp8_e4m3 with unit
+ * cache scales).  For every token t:
+ *     k_cache[loc[t], i] = e4m3(k[t, i]),  v_cache[loc[t], i] = e4m3(v[t, i])
+ * where e4m3(x) is the saturating round-to-nearest-even E4M3 code of x / 1 = x
+ * (the same rule as every other code; NaN stays NaN, +-infinity gives +-448).
+ *   k_bf16, v_bf16 : in, BF16 rows, row t at (element) offset t * row_stride;
+ *       width elements per row (all KV heads of the token, e.g. the K and V
+ *       column ranges of the fused QKV output, row_stride = its width).
+ *   loc            : in, int64 [T] cache slot of each token (device memory).
+ *   k_cache, v_cache : in/out, E4M3 codes, slot s at byte offset s * slot_stride;
+ *       the first width bytes of each written slot are replaced, nothing else.
+ *   num_slots      : slots in each cache.
+ * Requirements: width and row_stride multiples of 8, slot_stride a multiple of
+ * 16 and >= width, k/v/caches 16-byte and loc 8-byte aligned (MISALIGNED
+ * otherwise).  Distinct tokens should have distinct slots (with duplicates,
+ * which row a slot keeps is unspecified).  A token whose slot is outside
+ * [0, num_slots) is skipped on the device and FP8BQ_ERR_INDEX is recorded in
+ * the device status word (read with fp8bq_last_device_status).
+ */
+FP8BQ_API fp8bq_status fp8bq_kv_write_e4m3(const void *k_bf16, const void *v_bf16,
+                                           int64_t row_stride, int64_t T, int64_t width,
+                                           const int64_t *loc, uint8_t *k_cache,
+                                           uint8_t *v_cache, int64_t num_slots,
+                                           int64_t slot_stride, void *stream);
+
+/*
+ * SiLU-gated MLP product, quantized for the down projection (page
+ * "ProCreations/Nanbeige4.3-33B-FP8", introduction: dynamic per-token group-128
+ * activation quantization for every linear layer).  With gate = gu[:, :I] and
+ * up = gu[:, I:],
+ *     h = BF16( silu(gate) * up ),  silu(g) = g / (1 + exp(-g)),
+ * and (q_e4m3, s) = the group-128 quantization of h, exactly what
+ * fp8bq_quantize_act would produce from that BF16 h.  h itself differs from
+ * the exactly rounded silu(gate) * up by at most one BF16 step (the
+ * exponential is the hardware one).
+ *   gu_bf16 : in, BF16 [M, 2I] row-major.
+ *   q_e4m3  : out, E4M3 [M, I];  s : out, FP32 [M, I/128].
+ *   h_bf16  : out, optional BF16 [M, I] (NULL: h is not stored).
+ * I must be a multiple of 128; pointers 16-byte aligned.
+ */
+FP8BQ_API fp8bq_status fp8bq_silu_mul_quantize(const void *gu_bf16, int64_t M, int64_t I,
+                                               uint8_t *q_e4m3, float *s, void *h_bf16,
+                                               void *stream);
 
 /*
  * fp8bq_gemm without a workspace argument, for callers that cannot allocate

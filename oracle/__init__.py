@@ -73,6 +73,7 @@ def _load():
         lib.oracle_kv_write.argtypes = [P, P, I, I, I, P, I, I, P, P]
         lib.oracle_kv_write.restype = ctypes.c_int64
         lib.oracle_silu_mul.argtypes = [P, I, I, P]
+        lib.oracle_bf16_round_array.argtypes = [P, I, P]
         lib.oracle_bf16_round.restype = ctypes.c_uint16
         _lib = lib
         return lib
@@ -174,12 +175,10 @@ def linear_ref(x, qw, sw, rows=None) -> np.ndarray:
 
 def bf16_round(v: np.ndarray) -> np.ndarray:
     """Nearest-even BF16 bit patterns of FP64 values (one rounding, from the exact value)."""
-    v = np.asarray(v, dtype=np.float64)
-    lib = _load()
-    flat = v.reshape(-1)
-    out = np.fromiter((lib.oracle_bf16_round(float(t)) for t in flat), dtype=np.uint16,
-                      count=flat.size)
-    return out.reshape(v.shape)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    _load().oracle_bf16_round_array(_ptr(v), v.size, _ptr(out))
+    return out
 
 
 def kv_write(k, v, loc, k_cache: np.ndarray, v_cache: np.ndarray) -> int:

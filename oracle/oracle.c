@@ -362,3 +362,11 @@ void oracle_silu_mul(const uint16_t *gu, int64_t M, int64_t I, double *h)
         }
     }
 }
+
+/* oracle_bf16_round over an array. */
+void oracle_bf16_round_array(const double *v, int64_t n, uint16_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; i++)
+        out[i] = oracle_bf16_round(v[i]);
+}

@@ -16,9 +16,11 @@ CANARY = 0xA5
 class Guarded:
     """A device tensor view with canary-filled guard bands on both sides."""
 
-    def __init__(self, shape, dtype, device="cuda"):
+    def __init__(self, shape, dtype, device="cuda", fill=None):
         nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
         self.raw = torch.full((nbytes + 2 * GUARD,), CANARY, dtype=torch.uint8, device=device)
+        if fill is not None:
+            self.raw[GUARD:GUARD + nbytes].fill_(fill)
         self.t = self.raw[GUARD:GUARD + nbytes].view(dtype).view(*shape)
         assert self.t.data_ptr() % 16 == 0
 

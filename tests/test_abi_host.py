@@ -22,7 +22,7 @@ from fp8_block_scaled_09_b200 import build as fp8bq_build
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
                       "fp8bq.h")
 
-OK, INVALID, SHAPE, MISALIGNED, WORKSPACE, CUDA, TIMEOUT, NODEV = range(8)
+OK, INVALID, SHAPE, MISALIGNED, WORKSPACE, CUDA, TIMEOUT, NODEV, INDEX = range(9)
 
 
 @pytest.fixture(scope="module")
@@ -34,13 +34,14 @@ def L():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(fp8bq_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(fp8bq_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_abi():
     names = declared_functions()
     for n in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
-              "fp8bq_workspace_size", "fp8bq_last_device_status", "fp8bq_status_string"):
+              "fp8bq_workspace_size", "fp8bq_last_device_status", "fp8bq_status_string",
+              "fp8bq_kv_write_e4m3", "fp8bq_silu_mul_quantize"):
         assert n in names
 
 
@@ -64,7 +65,7 @@ def test_only_the_abi_is_exported(L):
 
 
 def test_status_strings(L):
-    for code in range(8):
+    for code in range(9):
         assert len(fp8bq.status_string(code)) > 0
     assert fp8bq.status_string(99) == "unknown status"
     assert L.fp8bq_version() == 100
@@ -124,6 +125,33 @@ def test_linear_argument_errors(L):
     assert f(None, None, None, 0, 256, 256, None, None, 0, None) == OK
 
 
+def test_kv_write_argument_errors(L):
+    f = L.fp8bq_kv_write_e4m3
+    #        k     v     rs    T  W     loc   kc    vc    slots sstride
+    assert f(GOOD, GOOD, 1024, 0, 1024, None, None, None, 0, 1024, None) == OK      # T == 0
+    assert f(GOOD, GOOD, 1024, -1, 1024, GOOD, GOOD, GOOD, 8, 1024, None) == INVALID
+    assert f(GOOD, GOOD, 1000, 4, 1024, GOOD, GOOD, GOOD, 8, 1024, None) == INVALID  # row_stride < W
+    assert f(GOOD, GOOD, 1024, 4, 1024, GOOD, GOOD, GOOD, 8, 1000, None) == INVALID  # slot < W
+    assert f(GOOD, GOOD, 1028, 4, 1020, GOOD, GOOD, GOOD, 8, 1024, None) == SHAPE    # W % 8
+    assert f(GOOD, GOOD, 1028, 4, 1024, GOOD, GOOD, GOOD, 8, 1024, None) == SHAPE    # stride % 8
+    assert f(GOOD, GOOD, 1024, 4, 1024, GOOD, GOOD, GOOD, 8, 1032, None) == SHAPE    # slot % 16
+    assert f(None, GOOD, 1024, 4, 1024, GOOD, GOOD, GOOD, 8, 1024, None) == INVALID
+    assert f(GOOD, GOOD, 1024, 4, 1024, None, GOOD, GOOD, 8, 1024, None) == INVALID
+    assert f(ODD, GOOD, 1024, 4, 1024, GOOD, GOOD, GOOD, 8, 1024, None) == MISALIGNED
+    assert f(GOOD, GOOD, 1024, 4, 1024, P(0x10004), GOOD, GOOD, 8, 1024, None) == MISALIGNED
+
+
+def test_silu_mul_quantize_argument_errors(L):
+    f = L.fp8bq_silu_mul_quantize
+    assert f(GOOD, 4, 100, GOOD, GOOD, None, None) == SHAPE     # I % 128
+    assert f(GOOD, -1, 128, GOOD, GOOD, None, None) == SHAPE
+    assert f(None, 0, 128, None, None, None, None) == OK         # M == 0
+    assert f(None, 4, 128, GOOD, GOOD, None, None) == INVALID
+    assert f(GOOD, 4, 128, GOOD, None, None, None) == INVALID
+    assert f(GOOD, 4, 128, ODD, GOOD, None, None) == MISALIGNED
+    assert f(GOOD, 4, 128, GOOD, GOOD, ODD, None) == MISALIGNED  # optional h, if given
+
+
 def test_workspace_sizes(L):
     g = lambda M, N, K: fp8bq.workspace_size(fp8bq.OP_GEMM, M, N, K)
     lin = lambda M, N, K: fp8bq.workspace_size(fp8bq.OP_LINEAR, M, N, K)
@@ -152,6 +180,8 @@ def test_valid_call_without_device_reports_no_device(L):
     assert L.fp8bq_quantize_act(GOOD, 4, 128, GOOD, GOOD, None) == NODEV
     assert L.fp8bq_last_device_status(None) == NODEV
     assert L.fp8bq_selftest_timeout(20000, None) == NODEV
+    assert L.fp8bq_kv_write_e4m3(GOOD, GOOD, 1024, 4, 1024, GOOD, GOOD, GOOD, 8, 1024, None) == NODEV
+    assert L.fp8bq_silu_mul_quantize(GOOD, 4, 128, GOOD, GOOD, None, None) == NODEV
 
 
 def test_selftest_limit_is_validated_on_the_host(L):
