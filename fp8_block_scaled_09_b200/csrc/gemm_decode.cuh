@@ -78,7 +78,7 @@ __host__ __device__ constexpr int token_tile(int64_t M) {
 
 // Units per ring slot / barrier / TMEM group, by token tile.
 __host__ __device__ constexpr int step_units_of(int /*MT*/) { return 2; }
-constexpr int kMaxRingUnits = 12;   // ring slots x units per slot, at most
+constexpr int kMaxRingUnits = 8;    // ring slots x units per slot, at most (measured: 8 beats 4, 6 ~ 8, 10 and 12 lose 2-4% on the decode step)
 constexpr int kMinStages = 2;
 constexpr int kMaxSmem = 227 * 1024;
 
