@@ -74,6 +74,12 @@ def _load():
         lib.oracle_kv_write.restype = ctypes.c_int64
         lib.oracle_silu_mul.argtypes = [P, I, I, P]
         lib.oracle_bf16_round_array.argtypes = [P, I, P]
+        lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e2m1_decode.restype = ctypes.c_double
+        lib.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e2m1_encode.restype = ctypes.c_uint8
+        lib.oracle_nvfp4_quantize.argtypes = [P, I, I, P, P, P]
+        lib.oracle_nvfp4_gemm_ref.argtypes = [P, P, I, I, P, P, ctypes.c_float, I, P]
         lib.oracle_bf16_round.restype = ctypes.c_uint16
         _lib = lib
         return lib
@@ -223,3 +229,42 @@ def _bf16_strided(x) -> np.ndarray:
     a = np.asarray(x)
     assert a.dtype == np.uint16 and a.ndim == 2 and a.strides[1] == 2
     return a
+
+
+def e2m1_decode(code: int) -> float:
+    return float(_load().oracle_e2m1_decode(int(code)))
+
+
+def e2m1_encode(y: float) -> int:
+    return int(_load().oracle_e2m1_encode(float(y)))
+
+
+def nvfp4_quantize(w) -> tuple[np.ndarray, np.ndarray, float]:
+    """Plain min-max NVFP4 quantization of BF16 W [N, K]: (packed uint8 [N, K/2],
+    E4M3 block scales uint8 [N, K/16], global FP32 scale)."""
+    wb = _bf16_bits(w)
+    N, K = wb.shape
+    packed = np.empty((N, K // 2), dtype=np.uint8)
+    sb = np.empty((N, K // 16), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    _load().oracle_nvfp4_quantize(_ptr(wb), N, K, _ptr(packed), _ptr(sb), _ptr(g))
+    return packed, sb, float(g[0])
+
+
+def nvfp4_gemm_ref(x, packed: np.ndarray, sb: np.ndarray, g: float, rows=None) -> np.ndarray:
+    """FP64 X . dequant(W)^T for BF16 X [M, K] and NVFP4 W; rows of Y as in gemm_ref."""
+    xb = _bf16_bits(x)
+    M, K = xb.shape
+    N = packed.shape[0]
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    sb = np.ascontiguousarray(sb, dtype=np.uint8)
+    if rows is None:
+        r = None
+        n_rows = M
+    else:
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = r.size
+    y = np.empty((n_rows, N), dtype=np.float64)
+    _load().oracle_nvfp4_gemm_ref(_ptr(xb), _ptr(r) if r is not None else None, n_rows, K,
+                                  _ptr(packed), _ptr(sb), ctypes.c_float(g), N, _ptr(y))
+    return y

@@ -370,3 +370,119 @@ void oracle_bf16_round_array(const double *v, int64_t n, uint16_t *out)
     for (int64_t i = 0; i < n; i++)
         out[i] = oracle_bf16_round(v[i]);
 }
+
+/*
+ * NVFP4 weight-only format with BF16 activations (page
+ * "ProCreations/Nanbeige4.3-33B-NVFP4-A16", the recipe paragraph: FP4 E2M1
+ * weights in groups of 16 with E4M3 block scales and a global weight scale;
+ * activations stay BF16).  A weight is
+ *     w = e2m1(q) * e4m3(sb) * g
+ * with q the 4-bit code, sb the E4M3 code of its 16-element group (16
+ * consecutive k of one row) and g one FP32 scale per tensor.
+ *
+ * E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit; magnitudes
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+ */
+double oracle_e2m1_decode(uint8_t code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -v : v;
+}
+
+/* nearest E2M1 value, ties to the even mantissa, magnitudes above 6 -> 6 */
+uint8_t oracle_e2m1_encode(float y)
+{
+    uint8_t sign = signbit(y) ? 0x8 : 0x0;
+    double a = fabs((double)y);
+    /* grid of the 8 magnitudes; between neighbours pick the nearer, ties to even m */
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    if (!(a < 6.0))
+        return sign | 0x7; /* saturate (NaN is outside the contract) */
+    int best = 0;
+    for (int c = 1; c < 8; c++) {
+        double d_best = fabs(a - mag[best]), d = fabs(a - mag[c]);
+        if (d < d_best || (d == d_best && (c & 1) == 0 && (best & 1) == 1))
+            best = c;
+    }
+    return sign | (uint8_t)best;
+}
+
+/*
+ * Plain min-max NVFP4 quantization of W [N, K] (BF16 bits), the reading taken
+ * here (the page's own scales come from a data-driven search, which needs
+ * calibration data):
+ *   g   = fl32(amax(W) / 2688)            (2688 = 6 * 448; 1 if W is all zero)
+ *   sb  = E4M3_RNE_sat(fl32(amax_group / fl32(6 * g)))
+ *   sig = fl32(e4m3(sb) * g)
+ *   q   = E2M1_RNE_sat(fl32(w / sig))       (0 when sig is 0)
+ * packed: [N, K/2] bytes, element 2j in the low nibble, 2j+1 in the high one;
+ * sb: [N, K/16] E4M3 codes; *g_out: the global scale.
+ */
+void oracle_nvfp4_quantize(const uint16_t *w, int64_t N, int64_t K, uint8_t *packed, uint8_t *sb,
+                           float *g_out)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < N * K; i++) {
+        float a = fabsf(bf16_bits_to_float(w[i]));
+        if (a > amax)
+            amax = a;
+    }
+    float g = amax == 0.0f ? 1.0f : amax / 2688.0f;
+    float six_g = 6.0f * g;
+    *g_out = g;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t b = 0; b < K / 16; b++) {
+            const uint16_t *wb = w + n * K + b * 16;
+            float ab = 0.0f;
+            for (int i = 0; i < 16; i++) {
+                float a = fabsf(bf16_bits_to_float(wb[i]));
+                if (a > ab)
+                    ab = a;
+            }
+            uint8_t code = oracle_e4m3_encode(ab / six_g);
+            sb[n * (K / 16) + b] = code;
+            float sig = (float)oracle_e4m3_decode(code) * g;
+            for (int i = 0; i < 16; i += 2) {
+                uint8_t lo = 0, hi = 0;
+                if (sig != 0.0f) {
+                    lo = oracle_e2m1_encode(bf16_bits_to_float(wb[i]) / sig);
+                    hi = oracle_e2m1_encode(bf16_bits_to_float(wb[i + 1]) / sig);
+                }
+                packed[n * (K / 2) + (b * 16 + i) / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    }
+}
+
+/*
+ * Y_ref[m, n] = sum_k x[m, k] * e2m1(q[n, k]) * e4m3(sb[n, k/16]) * g in FP64,
+ * x BF16 [M, K]; rows of Y listed in `rows` (all when rows is NULL, n_rows = M).
+ */
+void oracle_nvfp4_gemm_ref(const uint16_t *x, const int64_t *rows, int64_t n_rows, int64_t K,
+                           const uint8_t *packed, const uint8_t *sb, float g, int64_t N, double *y)
+{
+#pragma omp parallel
+    {
+        double *wr = (double *)malloc(sizeof(double) * (size_t)K);
+#pragma omp for schedule(static)
+        for (int64_t n = 0; n < N; n++) {
+            for (int64_t k = 0; k < K; k++) {
+                uint8_t byte = packed[n * (K / 2) + k / 2];
+                uint8_t q = (k & 1) ? (byte >> 4) : (byte & 0xF);
+                wr[k] = oracle_e2m1_decode(q) * oracle_e4m3_decode(sb[n * (K / 16) + k / 16]) *
+                        (double)g;
+            }
+            for (int64_t r = 0; r < n_rows; r++) {
+                int64_t m = rows ? rows[r] : r;
+                const uint16_t *xm = x + m * K;
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; k++)
+                    acc += (double)bf16_bits_to_float(xm[k]) * wr[k];
+                y[r * N + n] = acc;
+            }
+        }
+        free(wr);
+    }
+}
