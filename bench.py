@@ -567,6 +567,44 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
         "unfused": "torch silu * up into BF16 h, then fp8bq.quantize_act(h): context only"}
     del gu, qh, sh, hb
 
+    # NVFP4 weight-only GEMM (A16), decode shapes: back-to-back graph replays over 4
+    # weight copies per shape (larger than L2), like the headline decode measurement
+    nv_rows = []
+    for name in ("qkv_m1", "o_proj_m1", "qkv_m8", "o_proj_m8"):
+        gshape = W.by_name(name)
+        w = gshape.make_w().to(dev)
+        copies = [fp8bq.nvfp4_quantize_weight(w) for _ in range(4)]
+        x = gshape.make_x().to(dev)
+        y = torch.empty((gshape.M, gshape.N), dtype=torch.bfloat16, device=dev)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for c in copies:
+                fp8bq.nvfp4_gemm_a16(x, *c, out=y)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for rep in range(2):
+                for c in copies:
+                    fp8bq.nvfp4_gemm_a16(x, *c, out=y)
+        for _ in range(3):
+            graph.replay()
+        with clocks:
+            t = events_ms(torch, lambda i: graph.replay(), iters)
+        us = t / (iters * 8) * 1e3
+        nbytes = (gshape.N * gshape.K // 2 + gshape.N * gshape.K // 16 + 4
+                  + gshape.M * gshape.K * 2 + gshape.M * gshape.N * 2)
+        nv_rows.append({"name": name, "M": gshape.M, "N": gshape.N, "K": gshape.K, "us": us,
+                        "gbs": nbytes / (us * 1e-6) / 1e9,
+                        "frac_hbm": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                        "algorithmic_bytes": nbytes})
+        del graph, copies, w, x, y
+    out["nvfp4_a16"] = {
+        "workload": "NVFP4 weight-only GEMM, BF16 activations: decode QKV / o_proj at M = 1, 8",
+        "rows": nv_rows,
+        "bytes": "E2M1 codes N*K/2 + E4M3 block scales N*K/16 + global scale + X BF16 + Y BF16",
+        "timing": "CUDA events around graph replays of 8 back-to-back launches over 4 weight copies"}
+
     rows = [pq]
     for g in (W.KPROJ_M16,) + W.DRAFTER_MLP + (W.LONG_O_PROJ,):
         rows.append(shape_result(g, True))
@@ -611,6 +649,12 @@ def run_profile_case(case: str) -> None:
         vc = torch.empty_like(kc)
         for _ in range(3):
             fp8bq.kv_write_e4m3(qkv[:, 7168:8192], qkv[:, 8192:], loc, kc, vc)
+    elif case == "nvfp4":
+        gs = W.by_name("o_proj_m8")
+        packed, sb, g = fp8bq.nvfp4_quantize_weight(gs.make_w().to(dev))
+        x = gs.make_x().to(dev)
+        for _ in range(3):
+            fp8bq.nvfp4_gemm_a16(x, packed, sb, g)
     elif case == "silu":
         gu = torch.randn((4096, 16384), device=dev).mul_(2).to(torch.bfloat16)
         for _ in range(3):
@@ -644,7 +688,8 @@ def main() -> None:
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--quick", action="store_true", help="decode set only (no prefill/workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=("decode", "midm", "prefill", "quantize", "kv", "silu"),
+    ap.add_argument("--only", choices=("decode", "midm", "prefill", "quantize", "kv", "silu",
+                                       "nvfp4"),
                     help="profiling case: run one kernel family a few times, print a short line")
     args = ap.parse_args()
 

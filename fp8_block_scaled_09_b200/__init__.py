@@ -15,6 +15,8 @@ Functions (names follow the C ABI without the ``fp8bq_`` prefix):
 * ``linear(x, qw, sw)``      -> BF16 [M, N], activation quantization fused into the call
 * ``kv_write_e4m3(k, v, loc, k_cache, v_cache)``  E4M3 unit-scale KV-cache write (in place)
 * ``silu_mul_quantize(gu)``  BF16 [M, 2I] gate|up -> (codes [M, I], FP32 [M, I/128])
+* ``nvfp4_quantize_weight(w)`` BF16 [N, K] -> (packed uint8 [N, K/2], E4M3 uint8 [N, K/16], FP32 [1])
+* ``nvfp4_gemm_a16(x, packed, sb, g)`` BF16 [M, K] x NVFP4 W -> BF16 [M, N]
 """
 from __future__ import annotations
 
@@ -28,7 +30,7 @@ __all__ = [
     "Fp8bqError", "lib", "quantize_act", "quantize_weight", "gemm", "gemm_noalloc", "linear",
     "workspace_size", "new_workspace", "workspace_init", "last_device_status",
     "launch_count", "status_string", "selftest_timeout", "OP_GEMM", "OP_LINEAR", "LIB_PATH",
-    "kv_write_e4m3", "silu_mul_quantize",
+    "kv_write_e4m3", "silu_mul_quantize", "nvfp4_quantize_weight", "nvfp4_gemm_a16",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bq.so")
@@ -71,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_selftest_timeout.argtypes = [ctypes.c_uint32, P]
         L.fp8bq_kv_write_e4m3.argtypes = [P, P, I, I, I, P, P, P, I, I, P]
         L.fp8bq_silu_mul_quantize.argtypes = [P, I, I, P, P, P, P]
+        L.fp8bq_nvfp4_quantize_weight.argtypes = [P, I, I, P, P, P, P]
+        L.fp8bq_nvfp4_gemm_a16.argtypes = [P, P, P, P, I, I, I, P, P]
         L.fp8bq_workspace_size.argtypes = [ctypes.c_int, I, I, I]
         L.fp8bq_workspace_size.restype = S
         L.fp8bq_workspace_init.argtypes = [P, S, P]
@@ -83,7 +87,8 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_version.restype = ctypes.c_int
         for name in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
                      "fp8bq_workspace_init", "fp8bq_last_device_status", "fp8bq_gemm_noalloc",
-                     "fp8bq_selftest_timeout", "fp8bq_kv_write_e4m3", "fp8bq_silu_mul_quantize"):
+                     "fp8bq_selftest_timeout", "fp8bq_kv_write_e4m3", "fp8bq_silu_mul_quantize",
+                     "fp8bq_nvfp4_quantize_weight", "fp8bq_nvfp4_gemm_a16"):
             getattr(L, name).restype = st
         _lib = L
         return L
@@ -280,3 +285,35 @@ def silu_mul_quantize(gu: torch.Tensor, q: torch.Tensor | None = None, s: torch.
     _check(lib().fp8bq_silu_mul_quantize(_ptr(gu), M, I, _ptr(q), _ptr(s), _ptr(h), _stream(gu)),
            "fp8bq_silu_mul_quantize")
     return q, s
+
+
+def nvfp4_quantize_weight(w: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """fp8bq_nvfp4_quantize_weight: BF16 W [N, K] -> (packed E2M1 uint8 [N, K/2], E4M3
+    block scales uint8 [N, K/16], global scale FP32 [1]), plain min-max."""
+    _need(w, torch.bfloat16, "w")
+    N, K = w.shape
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    sb = torch.empty((N, K // 16), dtype=torch.uint8, device=w.device)
+    g = torch.empty(1, dtype=torch.float32, device=w.device)
+    _check(lib().fp8bq_nvfp4_quantize_weight(_ptr(w), N, K, _ptr(packed), _ptr(sb), _ptr(g),
+                                             _stream(w)), "fp8bq_nvfp4_quantize_weight")
+    return packed, sb, g
+
+
+def nvfp4_gemm_a16(x: torch.Tensor, packed: torch.Tensor, sb: torch.Tensor, g: torch.Tensor,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp8bq_nvfp4_gemm_a16: BF16 X [M, K] times the NVFP4 weight (packed [N, K/2], sb
+    [N, K/16], g FP32 [1]) transposed -> BF16 [M, N]."""
+    _need(x, torch.bfloat16, "x")
+    _need(packed, torch.uint8, "packed")
+    sb = _codes(sb)
+    _need(sb, torch.uint8, "sb")
+    _need(g, torch.float32, "g")
+    M, K = x.shape
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    _check(lib().fp8bq_nvfp4_gemm_a16(_ptr(x), _ptr(packed), _ptr(sb), _ptr(g), M, N, K, _ptr(out),
+                                      _stream(x)), "fp8bq_nvfp4_gemm_a16")
+    return out

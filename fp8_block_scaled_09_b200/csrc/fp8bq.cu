@@ -12,6 +12,8 @@
 //   gemm, M > 128    -> prefill::gemm_prefill_kernel<256> (persistent tcgen05;
 //                       the CTA-pair kernel prefill2 is built but not dispatched)
 //   kv_write_e4m3    -> kv_write_e4m3_kernel (warp per K/V row, slot scatter)
+//   nvfp4_quantize_weight -> nvfp4 amax, quantize and global-scale kernels
+//   nvfp4_gemm_a16   -> nvfp4::nvfp4_gemm_a16_kernel (BF16 dequant + tcgen05 kind::f16)
 //   silu_mul_quantize-> silu_mul_quantize_kernel (half-warp per 128-channel group)
 //   linear           -> quantize_act into the workspace, then the gemm path; the
 //                       decode kernel then streams its first weight blocks while
@@ -31,6 +33,7 @@
 #include "gemm_prefill2.cuh"
 #include "ptx.cuh"
 #include "kv_cache.cuh"
+#include "nvfp4.cuh"
 #include "quantize.cuh"
 #include "silu_quant.cuh"
 
@@ -73,6 +76,7 @@ struct DeviceInfo {
     // co-resident decode clusters of each size 2..8 (one CTA per SM at full
     // shared memory); the decode plan only uses sizes whose clusters all fit
     int cluster_capacity[9] = {};
+    int nvfp4_cluster_capacity[9] = {};  // the same for the NVFP4 A16 GEMM
     int *status = nullptr;  // device address of g_status
     bool supported = false;
 };
@@ -186,6 +190,28 @@ const DeviceInfo *device_info() {
             cudaGetLastError();  // clear a failed query
             d.cluster_capacity[c] = n;
         }
+        if (cudaFuncSetAttribute(nvfp4::nvfp4_gemm_a16_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 nvfp4::Layout::kBytes) != cudaSuccess)
+            return;
+        for (int c = 2; c <= 8; ++c) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(static_cast<unsigned>(c));
+            cfg.blockDim = dim3(nvfp4::kNumThreads);
+            cfg.dynamicSmemBytes = nvfp4::Layout::kBytes;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = static_cast<unsigned>(c);
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, nvfp4::nvfp4_gemm_a16_kernel, &cfg) != cudaSuccess)
+                n = 0;
+            cudaGetLastError();
+            d.nvfp4_cluster_capacity[c] = n;
+        }
         if (cudaDeviceSynchronize() != cudaSuccess) return;
         d.supported = true;
     });
@@ -253,6 +279,23 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 
 // 2-D uint8 tensor map over a row-major [rows, cols] byte matrix, box
 // [box_rows, 128 bytes], 128-byte swizzle, zero fill out of bounds.
+// 2-D tensor map over a row-major [rows, cols] matrix of `type` (elem_bytes each),
+// box [box_rows, box_cols], zero fill out of bounds.
+bool make_tmap_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType type, int elem_bytes,
+                  int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows,
+                  CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * elem_bytes)};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t elem[2] = {1u, 1u};
+    std::memset(map, 0, sizeof(*map));
+    return enc(map, type, 2, const_cast<void *>(ptr), dims, strides, box, elem,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, uint32_t box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
@@ -535,6 +578,70 @@ fp8bq_status fp8bq_silu_mul_quantize(const void *gu_bf16, int64_t M, int64_t I, 
                             dim3(kSiluThreads), 0, static_cast<cudaStream_t>(stream),
                             static_cast<const uint4 *>(gu_bf16), M, I,
                             reinterpret_cast<uint2 *>(q_e4m3), s, static_cast<uint4 *>(h_bf16)));
+}
+
+fp8bq_status fp8bq_nvfp4_quantize_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *packed,
+                                         uint8_t *sb, float *g, void *stream) {
+    if (N <= 0 || K <= 0 || K % 16 != 0 || N > kMaxDim || K > kMaxDim || K > kMaxBytes / 2 / N)
+        return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    if (!w_bf16 || !packed || !sb || !g) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(w_bf16) || !aligned16(packed) || !aligned16(sb) ||
+        (reinterpret_cast<uintptr_t>(g) & 3u) != 0)
+        return FP8BQ_ERR_MISALIGNED;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n_vec = N * K / 8, groups = N * K / 16;
+    const int64_t cap = static_cast<int64_t>(d->sm_count) * 8;
+    unsigned int *gw = reinterpret_cast<unsigned int *>(g);
+    cudaError_t e = cudaMemsetAsync(g, 0, sizeof(float), st);
+    if (e == cudaSuccess)
+        e = launch(nvfp4::nvfp4_amax_kernel, dim3(static_cast<unsigned>(std::min((n_vec + 255) / 256, cap))),
+                   dim3(256), 0, st, static_cast<const uint4 *>(w_bf16), n_vec, gw);
+    if (e == cudaSuccess)
+        e = launch(nvfp4::nvfp4_quantize_kernel,
+                   dim3(static_cast<unsigned>(std::min((groups + 255) / 256, 2 * cap))), dim3(256), 0,
+                   st, static_cast<const uint4 *>(w_bf16), groups, static_cast<const unsigned int *>(gw),
+                   reinterpret_cast<uint2 *>(packed), sb);
+    if (e == cudaSuccess) e = launch(nvfp4::nvfp4_global_kernel, dim3(1), dim3(1), 0, st, gw);
+    return from_cuda(e);
+}
+
+fp8bq_status fp8bq_nvfp4_gemm_a16(const void *x_bf16, const uint8_t *packed, const uint8_t *sb,
+                                  const float *g, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                                  void *stream) {
+    if (M < 0 || N <= 0 || K <= 0 || N % 128 != 0 || K % nvfp4::BKU != 0 || M > kMaxDim ||
+        N > kMaxDim || K > kMaxDim || (M > 0 && K > kMaxBytes / 2 / M) || N / 128 > 65535)
+        return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return FP8BQ_OK;
+    if (!x_bf16 || !packed || !sb || !g || !y_bf16) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(sb) || !aligned16(y_bf16) ||
+        (reinterpret_cast<uintptr_t>(g) & 3u) != 0)
+        return FP8BQ_ERR_MISALIGNED;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    const int64_t NB = N / 128, KB = K / nvfp4::BKU, sms = d->sm_count;
+    int64_t S = 1;
+    if (NB <= sms) {
+        S = std::min<int64_t>(std::min<int64_t>(8, sms / NB), KB);
+        while (S >= 2 && NB > d->nvfp4_cluster_capacity[S]) --S;
+        S = std::max<int64_t>(S, 1);
+    }
+    const int64_t mtiles = (M + nvfp4::MT - 1) / nvfp4::MT;
+    if (mtiles > 65535) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    CUtensorMap tw, ts, tx;
+    if (!make_tmap_2d(&tw, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&ts, sb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 16, 16, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tmap_2d(&tx, x_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, 64, nvfp4::MT,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return FP8BQ_ERR_CUDA;
+    return from_cuda(launch_clustered(
+        nvfp4::nvfp4_gemm_a16_kernel, dim3(static_cast<unsigned>(NB * S), static_cast<unsigned>(mtiles)),
+        dim3(nvfp4::kNumThreads), nvfp4::Layout::kBytes, static_cast<cudaStream_t>(stream),
+        S > 1 ? static_cast<unsigned>(S) : 1u, tw, ts, tx, g, static_cast<__nv_bfloat16 *>(y_bf16),
+        static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(S), d->status));
 }
 
 size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {

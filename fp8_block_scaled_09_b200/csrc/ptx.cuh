@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -202,6 +203,25 @@ __host__ __device__ constexpr uint32_t umma_idesc_e4m3(int m, int n) {
            | (0u << 7) | (0u << 10)                      // A, B format: E4M3
            | (static_cast<uint32_t>(n >> 3) << 17)       // N / 8
            | (static_cast<uint32_t>(m >> 4) << 24);      // M / 16
+}
+
+// Instruction descriptor: BF16 x BF16 -> FP32, both operands K-major, dense.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int m, int n) {
+    return (1u << 4)                                     // D format: F32
+           | (1u << 7) | (1u << 10)                      // A, B format: BF16
+           | (static_cast<uint32_t>(n >> 3) << 17)       // N / 8
+           | (static_cast<uint32_t>(m >> 4) << 24);      // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T over K = 16 (one BF16 MMA, issued by one thread).
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T over K = 32 (one FP8 MMA, issued by one thread).
@@ -409,6 +429,29 @@ __device__ __forceinline__ void umma_commit_pair_multicast(uint64_t *bar, uint16
 
 // Two binary32 values -> two E4M3 codes (round to nearest even, saturating at
 // +-448), `lo` in the low byte.
+// Eight floats -> eight E2M1 codes (nearest, ties to even, saturating at +-6),
+// element i in nibble i of the result (element 0 in the low nibble).
+__device__ __forceinline__ uint32_t e2m1x8_satfinite(const float (&v)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
+// Value of an E4M3 code (exact, through the f16 conversion).
+__device__ __forceinline__ float e4m3_to_float(uint32_t code) {
+    uint32_t h2;
+    const uint16_t c = static_cast<uint16_t>(code & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
 __device__ __forceinline__ uint16_t e4m3x2_satfinite(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));

@@ -181,6 +181,40 @@ FP8BQ_API fp8bq_status fp8bq_silu_mul_quantize(const void *gu_bf16, int64_t M, i
                                                void *stream);
 
 /*
+ * NVFP4 weight-only format with BF16 activations (page
+ * "ProCreations/Nanbeige4.3-33B-NVFP4-A16", recipe paragraph: FP4 E2M1 weights
+ * in groups of 16 with E4M3 block scales and a global weight scale; activations
+ * BF16).  A weight is w[n, k] = e2m1(q[n, k]) * e4m3(sb[n, k/16]) * g.
+ * Layout: packed [N, K/2] bytes, element 2j in the low nibble and 2j+1 in the
+ * high nibble of byte j of its row; sb [N, K/16] E4M3 codes; g one FP32 value.
+ *
+ * fp8bq_nvfp4_quantize_weight: plain min-max quantization (the page's own
+ * scales come from a data-driven search, which needs calibration data):
+ *   g  = fl32(amax(|W|) / 2688)   (2688 = 6 * 448; 1.0 when W is all zero)
+ *   sb = E4M3_RNE_sat(fl32(amax_group / fl32(6 g)))
+ *   q  = E2M1_RNE_sat(fl32(w / fl32(e4m3(sb) * g)))   (0 when that scale is 0)
+ *   w_bf16 : in, BF16 [N, K], K a multiple of 16.
+ *   packed : out, [N, K/2];  sb : out, [N, K/16];  g : out, one float (device).
+ * Codes, block scales and g are bit-exact with that definition.  Pointers
+ * 16-byte aligned (g: 4).  Three kernels and a 4-byte memset on `stream`.
+ */
+FP8BQ_API fp8bq_status fp8bq_nvfp4_quantize_weight(const void *w_bf16, int64_t N, int64_t K,
+                                                   uint8_t *packed, uint8_t *sb, float *g,
+                                                   void *stream);
+
+/*
+ * Y[m, n] = BF16( sum_k x[m, k] * w[n, k] ) for BF16 X [M, K] and an NVFP4 W
+ * [N, K] in the layout above; g is read from device memory (e.g. as written by
+ * fp8bq_nvfp4_quantize_weight).  N a multiple of 128, K a multiple of 256;
+ * pointers 16-byte aligned (g: 4).  No workspace.  Accuracy as fp8bq_gemm:
+ * |y - ref| <= 1e-2 |ref| + 2e-3 rms(ref) against the FP64 sum.  Built for
+ * decode-sized M; every 16 rows of M stream the weights once.
+ */
+FP8BQ_API fp8bq_status fp8bq_nvfp4_gemm_a16(const void *x_bf16, const uint8_t *packed,
+                                            const uint8_t *sb, const float *g, int64_t M,
+                                            int64_t N, int64_t K, void *y_bf16, void *stream);
+
+/*
  * fp8bq_gemm without a workspace argument, for callers that cannot allocate
  * device memory: code running where no allocator is reachable (an embedding
  * runtime that hands out only fixed buffers, or a context where cudaMalloc is

@@ -152,6 +152,21 @@ def test_silu_mul_quantize_argument_errors(L):
     assert f(GOOD, 4, 128, GOOD, GOOD, ODD, None) == MISALIGNED  # optional h, if given
 
 
+def test_nvfp4_argument_errors(L):
+    q = L.fp8bq_nvfp4_quantize_weight
+    assert q(GOOD, 128, 100, GOOD, GOOD, GOOD, None) == SHAPE    # K % 16
+    assert q(GOOD, 0, 128, GOOD, GOOD, GOOD, None) == SHAPE
+    assert q(None, 128, 128, GOOD, GOOD, GOOD, None) == INVALID
+    assert q(GOOD, 128, 128, GOOD, GOOD, P(0x10002), None) == MISALIGNED
+    f = L.fp8bq_nvfp4_gemm_a16
+    #        x     packed sb    g     M  N    K
+    assert f(GOOD, GOOD, GOOD, GOOD, 4, 128, 128, GOOD, None) == SHAPE     # K % 256
+    assert f(GOOD, GOOD, GOOD, GOOD, 4, 100, 256, GOOD, None) == SHAPE     # N % 128
+    assert f(None, None, None, None, 0, 128, 256, None, None) == OK         # M == 0
+    assert f(GOOD, GOOD, GOOD, None, 4, 128, 256, GOOD, None) == INVALID
+    assert f(ODD, GOOD, GOOD, GOOD, 4, 128, 256, GOOD, None) == MISALIGNED
+
+
 def test_workspace_sizes(L):
     g = lambda M, N, K: fp8bq.workspace_size(fp8bq.OP_GEMM, M, N, K)
     lin = lambda M, N, K: fp8bq.workspace_size(fp8bq.OP_LINEAR, M, N, K)
@@ -182,6 +197,8 @@ def test_valid_call_without_device_reports_no_device(L):
     assert L.fp8bq_selftest_timeout(20000, None) == NODEV
     assert L.fp8bq_kv_write_e4m3(GOOD, GOOD, 1024, 4, 1024, GOOD, GOOD, GOOD, 8, 1024, None) == NODEV
     assert L.fp8bq_silu_mul_quantize(GOOD, 4, 128, GOOD, GOOD, None, None) == NODEV
+    assert L.fp8bq_nvfp4_quantize_weight(GOOD, 128, 256, GOOD, GOOD, GOOD, None) == NODEV
+    assert L.fp8bq_nvfp4_gemm_a16(GOOD, GOOD, GOOD, GOOD, 4, 128, 256, GOOD, None) == NODEV
 
 
 def test_selftest_limit_is_validated_on_the_host(L):
