@@ -650,7 +650,7 @@ def run_profile_case(case: str) -> None:
         for _ in range(3):
             fp8bq.kv_write_e4m3(qkv[:, 7168:8192], qkv[:, 8192:], loc, kc, vc)
     elif case == "nvfp4":
-        gs = W.by_name("o_proj_m8")
+        gs = W.by_name("o_proj_m1")
         packed, sb, g = fp8bq.nvfp4_quantize_weight(gs.make_w().to(dev))
         x = gs.make_x().to(dev)
         for _ in range(3):

@@ -13,7 +13,9 @@
 //                       the CTA-pair kernel prefill2 is built but not dispatched)
 //   kv_write_e4m3    -> kv_write_e4m3_kernel (warp per K/V row, slot scatter)
 //   nvfp4_quantize_weight -> nvfp4 amax, quantize and global-scale kernels
-//   nvfp4_gemm_a16   -> nvfp4::nvfp4_gemm_a16_kernel (BF16 dequant + tcgen05 kind::f16)
+//   nvfp4_gemm_a16   -> M <= 4: nvfp4::nvfp4_gemv_a16_kernel<1|2|4> (codes decoded in
+//                       registers, CUDA-core FMA); larger M: nvfp4::nvfp4_gemm_a16_kernel
+//                       (BF16 dequant into shared memory + tcgen05 kind::f16)
 //   silu_mul_quantize-> silu_mul_quantize_kernel (half-warp per 128-channel group)
 //   linear           -> quantize_act into the workspace, then the gemm path; the
 //                       decode kernel then streams its first weight blocks while
@@ -192,7 +194,16 @@ const DeviceInfo *device_info() {
         }
         if (cudaFuncSetAttribute(nvfp4::nvfp4_gemm_a16_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 nvfp4::Layout::kBytes) != cudaSuccess)
+                                 nvfp4::Layout::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(nvfp4::nvfp4_gemv_a16_kernel<1>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 nvfp4::GemvLayout<1>::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(nvfp4::nvfp4_gemv_a16_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 nvfp4::GemvLayout<2>::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(nvfp4::nvfp4_gemv_a16_kernel<4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 nvfp4::GemvLayout<4>::kBytes) != cudaSuccess)
             return;
         for (int c = 2; c <= 8; ++c) {
             cudaLaunchConfig_t cfg = {};
@@ -630,6 +641,37 @@ fp8bq_status fp8bq_nvfp4_gemm_a16(const void *x_bf16, const uint8_t *packed, con
     const int64_t mtiles = (M + nvfp4::MT - 1) / nvfp4::MT;
     if (mtiles > 65535) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
     CUtensorMap tw, ts, tx;
+    if (M <= 4) {
+        // a handful of tokens: packed codes decoded in registers on the CUDA cores
+        const int MB = M <= 1 ? 1 : M <= 2 ? 2 : 4;
+        if (!make_tmap_2d(&tw, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_2d(&ts, sb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 16, 16, 128,
+                          CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !make_tmap_2d(&tx, x_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, nvfp4::BKU,
+                          static_cast<uint32_t>(MB), CU_TENSOR_MAP_SWIZZLE_NONE))
+            return FP8BQ_ERR_CUDA;
+        const dim3 grid(static_cast<unsigned>(NB * S)), block(nvfp4::kGemvThreads);
+        const unsigned cl = S > 1 ? static_cast<unsigned>(S) : 1u;
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        __nv_bfloat16 *yp = static_cast<__nv_bfloat16 *>(y_bf16);
+        const int iM = static_cast<int>(M), iN = static_cast<int>(N), iK = static_cast<int>(K),
+                  iS = static_cast<int>(S);
+        cudaError_t e;
+        if (MB == 1)
+            e = launch_clustered(nvfp4::nvfp4_gemv_a16_kernel<1>, grid, block,
+                                 nvfp4::GemvLayout<1>::kBytes, st, cl, tw, ts, tx, g, yp, iM, iN, iK,
+                                 iS, d->status);
+        else if (MB == 2)
+            e = launch_clustered(nvfp4::nvfp4_gemv_a16_kernel<2>, grid, block,
+                                 nvfp4::GemvLayout<2>::kBytes, st, cl, tw, ts, tx, g, yp, iM, iN, iK,
+                                 iS, d->status);
+        else
+            e = launch_clustered(nvfp4::nvfp4_gemv_a16_kernel<4>, grid, block,
+                                 nvfp4::GemvLayout<4>::kBytes, st, cl, tw, ts, tx, g, yp, iM, iN, iK,
+                                 iS, d->status);
+        return from_cuda(e);
+    }
     if (!make_tmap_2d(&tw, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_2d(&ts, sb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 16, 16, 128,

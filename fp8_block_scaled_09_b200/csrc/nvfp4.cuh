@@ -398,5 +398,213 @@ nvfp4_gemm_a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     }
 }
 
+
+// ---------------------------------------------------------------- GEMV (M <= 4)
+//
+// For a handful of tokens the tensor-core path above is bound by shared-memory
+// traffic (a 4 KB BF16 tile per 512 codes, written and read again).  This
+// kernel keeps the codes packed: each thread decodes its codes in registers
+// (hardware E2M1 -> f16 conversion, then f32) and multiplies them with the
+// activations on the CUDA cores, two k at a time (packed FP32 FMA), per
+// 16-element group then times the block scale.  Same units, TMA ring, split
+// and cluster reduction as the tensor-core kernel.
+//   warp 0      TMA producer (codes 128-byte swizzled, scales, activation tile)
+//   warp 1      converts each stage's BF16 activation tile to FP32 [MB][256]
+//   warps 2..17 thread (row r = t mod 128, 64-k quarter q = t / 128): 64 codes
+//               of its row per unit; a warp's lanes are 32 rows at the same k,
+//               so the activation reads are shared-memory broadcasts.
+template <int MB>
+struct GemvLayout {
+    static constexpr int kStages = 8;
+    static constexpr int kW = BNW * BKU / 2;             // 16 KB codes
+    static constexpr int kS = BNW * BKU / 16;            // 2 KB scales
+    static constexpr int kXb = 2048;                     // BF16 [MB][256] (<= 2 KB)
+    static constexpr int kXf = 4096;                     // FP32 [MB][256] (<= 4 KB)
+    static constexpr int kStage = kW + kS + kXb + kXf;   // 24 KB
+    static constexpr int kRedOff = kStages * kStage;     // [4][MB][128] FP32 quarter sums
+    static constexpr int kBarOff = kRedOff + 4 * MB * BNW * 4;
+    static constexpr int kNumBars = 3 * kStages;         // full, xready, empty
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kBytes = kMiscOff + 16 + 1024;
+};
+constexpr int kGemvComputeWarps = 16;
+constexpr int kGemvThreads = 32 * (2 + kGemvComputeWarps);  // 576
+
+template <int MB>
+__global__ void __launch_bounds__(kGemvThreads, 1)
+nvfp4_gemv_a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                      const __grid_constant__ CUtensorMap tmap_s,
+                      const __grid_constant__ CUtensorMap tmap_x, const float *__restrict__ g_ptr,
+                      __nv_bfloat16 *__restrict__ y, int M, int N, int K, int cluster_s,
+                      int *status) {
+    static_assert(MB == 1 || MB == 2 || MB == 4, "token count bucket");
+    using L = GemvLayout<MB>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+    uint64_t *xready = full + L::kStages;
+    uint64_t *empty = xready + L::kStages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KB = K / BKU;
+    const int S = cluster_s;
+    const int nb = static_cast<int>(blockIdx.x) / S, r = static_cast<int>(blockIdx.x) % S;
+    const int kb_begin = r * KB / S, kb_end = (r + 1) * KB / S;
+    const int n_units = kb_end - kb_begin;
+
+    allow_dependent_launch();
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < L::kStages; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&xready[st], 1);
+            mbar_init(&empty[st], kGemvComputeWarps);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tmap(&tmap_w);
+        prefetch_tmap(&tmap_s);
+        prefetch_tmap(&tmap_x);
+    }
+    __syncthreads();
+    grid_dependency_wait();
+
+    float acc[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) acc[m] = 0.0f;
+    const int ct = threadIdx.x - 64;  // compute thread 0..511
+    const int row = ct & 127, q = ct >> 7;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t evict_first = l2_policy_evict_first();
+            uint32_t stage = 0, phase = 0;
+            for (int u = 0; u < n_units; ++u) {
+                if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) break;
+                const int kb = kb_begin + u;
+                uint8_t *st = smem + stage * L::kStage;
+                mbar_arrive_expect_tx(&full[stage], L::kW + L::kS + MB * BKU * 2);
+                tma_load_2d_hint(st, &tmap_w, &full[stage], kb * (BKU / 2), nb * BNW, evict_first);
+                tma_load_2d_hint(st + L::kW, &tmap_s, &full[stage], kb * (BKU / 16), nb * BNW,
+                                 evict_first);
+                tma_load_2d(st + L::kW + L::kS, &tmap_x, &full[stage], kb * BKU, 0);
+                if (++stage == L::kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        uint32_t stage = 0, phase = 0;
+        for (int u = 0; u < n_units; ++u) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, status)) break;
+            uint8_t *st = smem + stage * L::kStage;
+            const uint32_t *xb = reinterpret_cast<const uint32_t *>(st + L::kW + L::kS);
+            float2 *xf = reinterpret_cast<float2 *>(st + L::kW + L::kS + L::kXb);
+            for (int i = lane; i < MB * BKU / 2; i += 32) {  // BF16 pairs -> float pairs
+                const uint32_t w = xb[i];
+                xf[i] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xready[stage]);
+            if (++stage == L::kStages) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+    } else {
+        uint32_t stage = 0, phase = 0;
+        for (int u = 0; u < n_units; ++u) {
+            if (!mbar_wait(&xready[stage], phase, abort_flag, status)) break;
+            const uint8_t *st = smem + stage * L::kStage;
+            const uint4 *prow = reinterpret_cast<const uint4 *>(st + row * 128);
+            const uint4 p0 = prow[(2 * q) ^ (row & 7)];
+            const uint4 p1 = prow[(2 * q + 1) ^ (row & 7)];
+            const uint32_t sc = *reinterpret_cast<const uint32_t *>(st + L::kW + row * 16 + 4 * q);
+            const float *xf = reinterpret_cast<const float *>(st + L::kW + L::kS + L::kXb);
+            const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {  // 16-element groups, one block scale each
+                float2 part[MB];
+#pragma unroll
+                for (int m = 0; m < MB; ++m) part[m] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {  // two code words of 8
+                    const uint32_t w = pw[2 * g + h];
+                    const int k0 = 64 * q + 16 * g + 8 * h;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {  // bytes: elements k0 + 2b, k0 + 2b + 1
+                        const float2 wv = e2m1x2_to_float2(w >> (8 * b));
+#pragma unroll
+                        for (int m = 0; m < MB; ++m) {
+                            const float2 xv = *reinterpret_cast<const float2 *>(xf + m * BKU + k0 + 2 * b);
+                            part[m] = ffma2(wv, xv, part[m]);
+                        }
+                    }
+                }
+                const float s = e4m3_to_float((sc >> (8 * g)) & 0xFFu);
+#pragma unroll
+                for (int m = 0; m < MB; ++m) acc[m] = fmaf(s, part[m].x + part[m].y, acc[m]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == L::kStages) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+        // quarter sums of this row -> shared memory
+        float *qs = reinterpret_cast<float *>(smem + L::kRedOff);
+#pragma unroll
+        for (int m = 0; m < MB; ++m) qs[(q * MB + m) * BNW + row] = acc[m];
+    }
+    __syncthreads();
+
+    // the CTA's partial [MB][128]: quarters summed in order, times g
+    const float g = __ldg(g_ptr);
+    float *part = reinterpret_cast<float *>(smem);  // ring memory is idle now
+    if (threadIdx.x < MB * BNW) {
+        const int m = threadIdx.x / BNW, n = threadIdx.x % BNW;
+        const float *qs = reinterpret_cast<const float *>(smem + L::kRedOff);
+        float v = 0.0f;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) v += qs[(qq * MB + m) * BNW + n];
+        v *= g;
+        if (S == 1) {
+            if (m < M) y[static_cast<int64_t>(m) * N + nb * BNW + n] = __float2bfloat16_rn(v);
+        } else {
+            part[m * BNW + n] = v;
+        }
+    }
+    if (S > 1) {
+        __syncwarp();
+        cluster_sync();
+        const uint32_t red = smem_addr(part);
+        const int items = M * (BNW / 4);
+        const int i0 = r * items / S, i1 = (r + 1) * items / S;
+        for (int item = i0 + static_cast<int>(threadIdx.x); item < i1; item += kGemvThreads) {
+            const int m = item / (BNW / 4), c4 = item % (BNW / 4);
+            const uint32_t off = static_cast<uint32_t>((m * BNW + 4 * c4) * 4);
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int p = 0; p < S; ++p) {
+                const float4 t = ld_shared_cluster_v4(map_to_cta(red + off, static_cast<uint32_t>(p)));
+                sum.x += t.x;
+                sum.y += t.y;
+                sum.z += t.z;
+                sum.w += t.w;
+            }
+            __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z, sum.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t *>(&lo);
+            pk.y = *reinterpret_cast<uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(y + static_cast<int64_t>(m) * N + nb * BNW + 4 * c4) = pk;
+        }
+        __syncwarp();
+        cluster_sync();
+    }
+}
+
 }  // namespace nvfp4
 }  // namespace fp8bq

@@ -444,6 +444,25 @@ __device__ __forceinline__ uint32_t e2m1x8_satfinite(const float (&v)[8]) {
     return r;
 }
 
+// Two E2M1 codes (one byte: element 0 in the low nibble) -> two floats (exact).
+__device__ __forceinline__ float2 e2m1x2_to_float2(uint32_t byte) {
+    uint32_t h2;
+    const uint16_t b = static_cast<uint16_t>(byte & 0xFFu);
+    asm("{\n\t.reg .b8 c;\n\tcvt.u8.u16 c, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}" : "=r"(h2) : "h"(b));
+    return make_float2(__half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu))),
+                       __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16))));
+}
+
+// d = a * b + c on float pairs (one packed FP32 instruction).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)),
+          "l"(*reinterpret_cast<const uint64_t *>(&c)));
+    return *reinterpret_cast<const float2 *>(&d);
+}
+
 // Value of an E4M3 code (exact, through the f16 conversion).
 __device__ __forceinline__ float e4m3_to_float(uint32_t code) {
     uint32_t h2;

@@ -69,19 +69,22 @@ def _run(M, N, K, seed):
     return x, packed, sb, g, y.t
 
 
+# M <= 4 runs the CUDA-core kernel (token buckets 1, 2, 4), larger M the tensor-core one
 @pytest.mark.parametrize("M,N,K", [(1, 128, 256), (4, 384, 1024), (16, 1024, 7168),
                                    (7, 640, 2048), (1, 9216, 7168), (8, 7168, 7168),
-                                   (33, 256, 512), (3, 20480, 256)])
+                                   (33, 256, 512), (3, 20480, 256), (2, 9216, 7168),
+                                   (2, 128, 21504), (3, 1024, 7168)])
 def test_nvfp4_gemm_a16_matches_oracle(M, N, K):
     x, packed, sb, g, y = _run(M, N, K, 50 + M)
     _check(bf16_to_f64(y), oracle.nvfp4_gemm_ref(x, packed, sb, g))
 
 
-def test_nvfp4_gemm_a16_exact_regime_bit_exact():
+@pytest.mark.parametrize("M", [1, 3, 5])
+def test_nvfp4_gemm_a16_exact_regime_bit_exact(M):
     # small-integer activations and power-of-two block scales: every partial sum
     # is exact in FP32, so the output is the BF16 rounding of the exact value
-    rng = np.random.default_rng(9)
-    M, N, K = 5, 256, 512
+    rng = np.random.default_rng(9 + M)
+    N, K = 256, 512
     x = torch.from_numpy(rng.integers(-3, 4, (M, K)).astype(np.float32)).to(torch.bfloat16)
     packed = rng.integers(0, 256, (N, K // 2)).astype(np.uint8)
     sb = rng.choice(np.array([0x30, 0x38, 0x40], np.uint8), size=(N, K // 16))  # 0.5, 1, 2
@@ -94,10 +97,11 @@ def test_nvfp4_gemm_a16_exact_regime_bit_exact():
     assert np.array_equal(got, oracle.bf16_round(ref))
 
 
-def test_nvfp4_gemm_a16_every_code_and_sign():
-    # each row of W cycles through all 16 E2M1 codes: the dequantization table
-    # (magnitudes and signs) is exercised against the oracle for every code
-    M, N, K = 2, 128, 256
+@pytest.mark.parametrize("M", [2, 6])
+def test_nvfp4_gemm_a16_every_code_and_sign(M):
+    # each row of W cycles through all 16 E2M1 codes: the code decoding of both
+    # kernels (magnitudes, signs, nibble order) is checked against the oracle
+    N, K = 128, 256
     codes = (np.arange(N * K) % 16).astype(np.uint8).reshape(N, K)
     packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
     sb = np.full((N, K // 16), 0x38, np.uint8)
