@@ -88,7 +88,9 @@ def test_gemm_mid_m_decode_path(M, N, K):
     check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
 
 
-PREFILL_SHAPES = [(129, 384, 1024), (255, 1152, 512),
+# M > 128 (the 129..256 rows of the mid-size range included) runs on the prefill kernel
+PREFILL_SHAPES = [(129, 384, 1024), (200, 2048, 7168), (255, 1152, 512), (256, 1024, 1024),
+                  (255, 9216, 256), (300, 1152, 512),
                   (1000, 512, 896), (300, 128, 7168), (2048, 2048, 384)]
 
 
@@ -145,7 +147,7 @@ def test_gemm_identity_weight_closed_form():
     check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
 
 
-@pytest.mark.parametrize("M", [8, 96, 600])
+@pytest.mark.parametrize("M", [8, 96, 200, 600])
 def test_gemm_deterministic(M):
     _, qa, sa, qw, sw = operands(M, 1024, 7168, 7)
     y1 = run_gemm(qa, sa, qw, sw).cpu()
@@ -165,7 +167,8 @@ def test_gemm_empty_m_is_noop():
 # ------------------------------------------------------------------ fused linear
 
 @pytest.mark.parametrize("M,N,K", [(1, 1024, 7168), (16, 1024, 7168), (5, 384, 640),
-                                   (33, 256, 1024), (128, 1152, 7168), (700, 384, 7168)])
+                                   (33, 256, 1024), (128, 1152, 7168), (192, 640, 2048),
+                                   (700, 384, 7168)])
 def test_linear_matches_oracle_and_unfused_path(M, N, K):
     x, qa, sa, qw, sw = operands(M, N, K, 300 + M)
     xd = x.cuda()
