@@ -166,9 +166,16 @@ def test_gemm_empty_m_is_noop():
 
 # ------------------------------------------------------------------ fused linear
 
-@pytest.mark.parametrize("M,N,K", [(1, 1024, 7168), (16, 1024, 7168), (5, 384, 640),
-                                   (33, 256, 1024), (128, 1152, 7168), (192, 640, 2048),
-                                   (700, 384, 7168)])
+# decode-sized M on every plan of the decode kernel (cluster split with S = 8,
+# 2, 1; stream-K with K ranges that wrap around K within a CTA; K so long that
+# the scale table takes most of the shared memory), and larger M.
+LINEAR_SHAPES = [(1, 1024, 7168), (16, 1024, 7168), (5, 384, 640), (1, 9216, 7168),
+                 (8, 7168, 7168), (17, 1152, 512), (32, 2048, 2048), (31, 640, 7168),
+                 (4, 19200, 512), (3, 32768, 256), (12, 16384, 1024), (20, 256, 128000),
+                 (33, 256, 1024), (128, 1152, 7168), (192, 640, 2048), (700, 384, 7168)]
+
+
+@pytest.mark.parametrize("M,N,K", LINEAR_SHAPES)
 def test_linear_matches_oracle_and_unfused_path(M, N, K):
     x, qa, sa, qw, sw = operands(M, N, K, 300 + M)
     xd = x.cuda()
