@@ -407,9 +407,19 @@ size_t act_ws_bytes(int64_t M, int64_t K) { return round256(M * K) + round256(M 
 
 // ---------------------------------------------------------------- launches
 
+// Up to this many groups (M <= 128 at K = 7168) the shared-memory-free
+// quantizer runs instead of the bulk-copy one.
+constexpr int64_t kSmallActMaxGroups = 8192;
+
 cudaError_t launch_quantize_act(const DeviceInfo &d, const void *x, int64_t M, int64_t K,
                                 uint8_t *q, float *sa, cudaStream_t st) {
     const int64_t groups = M * (K / 128);
+    if (groups <= kSmallActMaxGroups)
+        return launch(quantize_act_small_kernel,
+                      dim3(static_cast<unsigned>((groups + kSmallActGroupsPerCta - 1) /
+                                                 kSmallActGroupsPerCta)),
+                      dim3(kSmallActThreads), 0, st, static_cast<const uint4 *>(x), groups,
+                      reinterpret_cast<uint2 *>(q), sa);
     const int64_t chunks = (groups + kActChunkGroups - 1) / kActChunkGroups;
     const int64_t max_ctas = static_cast<int64_t>(d.sm_count) * kActCtasPerSm;
     const int blocks = static_cast<int>(std::min(chunks, max_ctas));

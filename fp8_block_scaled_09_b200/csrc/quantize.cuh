@@ -149,6 +149,33 @@ quantize_act_kernel(const uint8_t *__restrict__ x, int64_t num_groups, uint2 *__
     }
 }
 
+// Small activations (decode batches): one 16-lane team per group, each lane
+// one 16-byte load straight from global memory.  With no shared memory and
+// 256 threads its CTAs fit on an SM beside a running decode GEMM CTA, so the
+// kernel is resident, and past its dependency wait, as soon as the previous
+// kernel completes.
+constexpr int kSmallActThreads = 256;
+constexpr int kSmallActGroupsPerCta = kSmallActThreads / 16;
+
+__global__ void __launch_bounds__(kSmallActThreads)
+quantize_act_small_kernel(const uint4 *__restrict__ x, int64_t num_groups, uint2 *__restrict__ q,
+                          float *__restrict__ sa) {
+    grid_dependency_wait();
+    allow_dependent_launch();
+    const int64_t g = static_cast<int64_t>(blockIdx.x) * kSmallActGroupsPerCta + (threadIdx.x >> 4);
+    const int sub = threadIdx.x & 15;
+    const bool ok = g < num_groups;
+    const uint4 v = ok ? x[g * 16 + sub] : make_uint4(0, 0, 0, 0);
+    uint32_t m = amax_bits8(v);
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    const float scale = scale_from_amax_bits(m);
+    if (ok) {
+        q[g * 16 + sub] = encode8(v, scale);
+        if (sub == 0) sa[g] = scale;
+    }
+}
+
 // ------------------------------------------------------------------ weights
 
 // One CTA per 128x128 block: 256 threads, each holding 8 of the block's 2048
