@@ -64,9 +64,10 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kPrefillBN = 256;
-// The CTA-pair prefill kernel is correct but, with two 256-column TMEM buffers,
-// its cross-SM release round trip per K chunk leaves the tensor pipe idle more
-// than the single-CTA kernel; it stays off until it has deeper buffering.
+// The CTA-pair prefill kernel is correct and, moving 2/3 of the operand bytes,
+// runs exactly as fast as the single-CTA kernel (both are bound by the
+// per-chunk TMEM hand-off, not by L2), and no faster under the power cap; the
+// single-CTA kernel stays the one dispatched.
 constexpr bool kUsePairPrefill = false;
 constexpr int64_t kDecodeMaxM = decode::kMaxMT;
 

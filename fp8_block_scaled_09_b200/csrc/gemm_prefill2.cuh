@@ -15,12 +15,17 @@
 //   warp 0      TMA producer (both CTAs): its A and B halves of each K chunk;
 //               the bytes complete on the even CTA's `full` barrier, which the
 //               even CTA's producer arms for both CTAs' bytes.
-//   warp 1      even CTA: MMA issuer (4 pair MMAs per K chunk into one of two
-//               TMEM buffers), commits multicast to both CTAs' `empty` and
-//               `tfull` barriers.  Odd CTA: TMEM allocation only.
+//   warps 1, 2  even CTA: MMA issuers, one per TMEM buffer (chunk i into buffer
+//               i mod 2 by warp 1 + (i mod 2), 4 pair MMAs per chunk), commits
+//               multicast to both CTAs' `empty` and `tfull` barriers.  Odd CTA:
+//               warp 1 allocates TMEM.
 //   warps 4-11  promotion + epilogue of the CTA's own 128 rows, exactly as in
 //               the single-CTA kernel; they release a TMEM buffer by arriving
-//               on the even CTA's `tempty` barrier (16 arrivals: 8 warps x 2).
+//               on the even CTA's `tempty` barrier (16 arrivals: 8 warps x 2),
+//               the odd CTA's warps with a relaxed remote arrive.
+// Measured equal to the single-CTA kernel (QKV 8192x9216x7168: 543 us on the
+// same GPU, 1.99 PFLOP/s) and not faster under the power cap; it is built and
+// off (see fp8bq.cu).
 #pragma once
 
 #include "gemm_prefill.cuh"
@@ -100,7 +105,7 @@ gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 2 * kPromoWarps);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&tmap_a);
@@ -153,14 +158,19 @@ gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     mbar_wait(&empty[i % kStages], static_cast<uint32_t>((i / kStages) & 1),
                               nullptr, status);
             }
-        } else if (warp == 1 && rank == 0) {
-            // ------------------------------------------------------------ pair MMA issuer
+        } else if ((warp == 1 || warp == 2) && rank == 0) {
+            // ------------------------------------------------------------ pair MMA issuers
             if (lane == 0) {
                 const uint32_t idesc = umma_idesc_e4m3(BM, BN);
-                uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
+                const uint32_t buf = static_cast<uint32_t>(warp - 1);
+                int64_t i = 0;
                 bool ok = true;
                 for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-                    for (int kb = 0; kb < KB; ++kb) {
+                    for (int kb = 0; kb < KB; ++kb, ++i) {
+                        if ((i & 1) != buf) continue;
+                        const uint32_t stage = static_cast<uint32_t>(i % kStages);
+                        const uint32_t phase = static_cast<uint32_t>((i / kStages) & 1);
+                        const uint32_t bphase = static_cast<uint32_t>((i >> 1) & 1);
                         // tempty gathers arrivals from both CTAs of the pair
                         if (!mbar_wait<true>(&tempty[buf], bphase ^ 1, abort_flag, status) ||
                             !mbar_wait(&full[stage], phase, abort_flag, status)) {
@@ -177,15 +187,9 @@ gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                                            umma_desc_sw128(b_addr + 32 * j), idesc, j > 0 ? 1u : 0u);
                         umma_commit_pair_multicast(&empty[stage], 0x3);
                         umma_commit_pair_multicast(&tfull[buf], 0x3);
-                        if (++stage == kStages) {
-                            stage = 0;
-                            phase ^= 1;
-                        }
-                        buf ^= 1;
-                        if (buf == 0) bphase ^= 1;
                     }
                 }
-                // every pair MMA issued has finished before TMEM is released
+                // every pair MMA either thread issued has finished before TMEM is released
                 umma_commit_pair_multicast(drain, 0x1);
                 mbar_wait(drain, 0, nullptr, status);
             }
@@ -243,7 +247,12 @@ gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     promote_chunk(taddr, scale, acc, last);
                     tc_fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_remote(buf ? tempty0_b1 : tempty0_b0);
+                    if (lane == 0) {
+                        if (rank == 0)
+                            mbar_arrive(&tempty[buf]);
+                        else
+                            mbar_arrive_remote_relaxed(buf ? tempty0_b1 : tempty0_b0);
+                    }
 #pragma unroll
                     for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(last[i], scale, acc[96 + i]);
                     buf ^= 1;
