@@ -456,7 +456,8 @@ cudaError_t launch_decode(const DeviceInfo &d, const uint8_t *qa, const float *s
 
 // early_weights: the decode kernel may request its first weight blocks before
 // its dependency wait (only valid right after this library's activation
-// quantizer, see gemm_decode.cuh).
+// quantizer, while the GEMM before it may still be running; see
+// gemm_decode.cuh).
 cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
                         const uint8_t *qw, const float *sw, int64_t M, int64_t N, int64_t K,
                         void *y, void *ws, cudaStream_t st, fp8bq_status *err,

@@ -246,9 +246,11 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     // Everything above overlaps the previous kernel in the stream.  With
     // early_weights the first kStages weight blocks are requested too: only
     // the linear layer sets it, when the previous kernel is its own activation
-    // quantizer, which writes activation codes and scales only and lets this
-    // kernel start after its own dependency wait.  Every other global access
-    // happens after the previous kernel has completed.
+    // quantizer, which writes activation codes and scales only.  No kernel of
+    // this library that writes weights lets its successor start before it
+    // completes, so every such kernel earlier in the stream has completed by
+    // the time this one starts.  Every other global access happens after the
+    // previous kernel has completed.
     // Units of step i: [u_begin + kStep i, min(u_end, u_begin + kStep (i + 1))).
     auto step_units = [&](int64_t i) {
         const int64_t left = u_end - (u_begin + kStep * i);

@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(256)
 nvfp4_quantize_kernel(const uint4 *__restrict__ w, int64_t groups, const unsigned int *g_word,
                       uint2 *__restrict__ packed, uint8_t *__restrict__ sb) {
     grid_dependency_wait();  // the amax pass
-    allow_dependent_launch();
+    // (no early start for the next kernel: this one writes weights)
     const float g = nvfp4_global_scale(*g_word);
     const float six_g = 6.0f * g;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < groups;

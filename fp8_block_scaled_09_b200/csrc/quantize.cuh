@@ -92,12 +92,13 @@ quantize_act_kernel(const uint8_t *__restrict__ x, int64_t num_groups, uint2 *__
         *abort_flag = 0;
         fence_barrier_init();
     }
+    // The next kernel (typically the GEMM this feeds) may start at once, so
+    // it can set up and stream its weights while this one runs: this kernel
+    // writes activation codes only, and no kernel of this library that writes
+    // weights lets its successor start before it completes.
+    allow_dependent_launch();
     __syncthreads();
     grid_dependency_wait();
-    // The next kernel may start only once this one has passed its own wait: a
-    // GEMM that streams weights early then never overtakes the kernel that
-    // may have produced them.
-    allow_dependent_launch();
 
     if (warp == kActConsumerWarps) {
         // ------------------------------------------------------------ producer
@@ -160,8 +161,8 @@ constexpr int kSmallActGroupsPerCta = kSmallActThreads / 16;
 __global__ void __launch_bounds__(kSmallActThreads)
 quantize_act_small_kernel(const uint4 *__restrict__ x, int64_t num_groups, uint2 *__restrict__ q,
                           float *__restrict__ sa) {
+    allow_dependent_launch();  // as in quantize_act_kernel
     grid_dependency_wait();
-    allow_dependent_launch();
     const int64_t g = static_cast<int64_t>(blockIdx.x) * kSmallActGroupsPerCta + (threadIdx.x >> 4);
     const int sub = threadIdx.x & 15;
     const bool ok = g < num_groups;
@@ -186,7 +187,8 @@ __global__ void __launch_bounds__(kWeightThreads)
 quantize_weight_kernel(const uint16_t *__restrict__ w, int64_t K, uint8_t *__restrict__ q,
                        float *__restrict__ sw) {
     __shared__ uint32_t warp_max[kWeightThreads / 32];
-    allow_dependent_launch();
+    // This kernel writes weights, so it never lets the next kernel start
+    // early: a decode GEMM may read its weights before its dependency wait.
     grid_dependency_wait();
     const int64_t bj = blockIdx.x;  // K block
     const int64_t bi = blockIdx.y;  // N block

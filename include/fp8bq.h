@@ -129,6 +129,10 @@ FP8BQ_API fp8bq_status fp8bq_gemm(const uint8_t *qa, const float *sa, const uint
  *   x_bf16 : in, BF16 [M, K]; qw / sw / y_bf16 as in fp8bq_gemm
  *   workspace : at least fp8bq_workspace_size(FP8BQ_OP_LINEAR, M, N, K) bytes,
  *               same state rule as fp8bq_gemm.
+ * On the decode path the call starts reading qw / sw while earlier kernels in
+ * the stream may still be running (programmatic dependent launch).  This is
+ * safe against this library's weight quantizers, which never let a successor
+ * start early; qw / sw must not be written by a foreign kernel that does.
  */
 FP8BQ_API fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const float *sw, int64_t M,
                           int64_t N, int64_t K, void *y_bf16, void *workspace, size_t ws_bytes,
