@@ -191,6 +191,50 @@ def test_linear_matches_oracle_and_unfused_path(M, N, K):
     assert torch.equal(y.t.view(torch.int16), y2.view(torch.int16))
 
 
+# ------------------------------------------------------------------ stream order
+
+def test_weights_quantized_right_before_the_linear():
+    # The decode linear requests weight blocks before its dependency wait.  The
+    # weight quantizer just before it on the same stream never lets its
+    # successor start early, so the linear must see the new weights, not the
+    # zeros the buffers held before.
+    M, N, K = 4, 9216, 7168
+    x = workloads.activation(M, K, 910, outliers=7)
+    w = workloads.weight(N, K, 911)
+    qw_ref, sw_ref = oracle.quantize_weight(w)
+    ref = oracle.linear_ref(x, qw_ref, sw_ref)
+    xd, wd = x.cuda(), w.cuda()
+    ws = fp8bq.new_workspace(fp8bq.OP_LINEAR, M, N, K, "cuda")
+    for _ in range(3):
+        qw = torch.zeros((N, K), dtype=torch.uint8, device="cuda")
+        sw = torch.zeros((N // 128, K // 128), dtype=torch.float32, device="cuda")
+        torch.cuda.synchronize()
+        fp8bq.quantize_weight(wd, qw, sw)
+        y = fp8bq.linear(xd, qw, sw, workspace=ws)
+        torch.cuda.synchronize()
+        check(bf16_to_f64(y), ref)
+
+
+@pytest.mark.parametrize("M", [8, 200])
+def test_linear_chain_reads_the_previous_output(M):
+    # Each layer's input is the previous layer's output, all launched back to
+    # back with one shared workspace and no host synchronisation: every
+    # activation read and workspace write must wait for the kernels before it.
+    K, layers = 1024, 6
+    x0 = workloads.activation(M, K, 920)
+    weights = [oracle.quantize_weight(workloads.weight(K, K, 921 + i)) for i in range(layers)]
+    ws = fp8bq.new_workspace(fp8bq.OP_LINEAR, M, K, K, "cuda")
+    cur, outs = x0.cuda(), []
+    for qw, sw in weights:
+        cur = fp8bq.linear(cur, to_dev_codes(qw), to_dev_f32(sw), workspace=ws)
+        outs.append(cur)
+    torch.cuda.synchronize()
+    prev = x0
+    for (qw, sw), y in zip(weights, outs):
+        check(bf16_to_f64(y), oracle.linear_ref(prev, qw, sw))
+        prev = y.cpu()
+
+
 def test_linear_kproj_workload_with_zero_row():
     g = workloads.KPROJ_M16
     x = g.make_x()
