@@ -13,7 +13,7 @@
 //                       the CTA-pair kernel prefill2 is built but not dispatched)
 //   kv_write_e4m3    -> kv_write_e4m3_kernel (warp per K/V row, slot scatter)
 //   nvfp4_quantize_weight -> nvfp4 amax, quantize and global-scale kernels
-//   nvfp4_gemm_a16   -> M <= 4: nvfp4::nvfp4_gemv_a16_kernel<1|2|4> (codes decoded in
+//   nvfp4_gemm_a16   -> M <= 2: nvfp4::nvfp4_gemv_a16_kernel<1|2> (codes decoded in
 //                       registers, CUDA-core FMA); larger M: nvfp4::nvfp4_gemm_a16_kernel
 //                       (BF16 dequant into shared memory + tcgen05 kind::f16)
 //   silu_mul_quantize-> silu_mul_quantize_kernel (half-warp per 128-channel group)
@@ -201,10 +201,7 @@ const DeviceInfo *device_info() {
                                  nvfp4::GemvLayout<1>::kBytes) != cudaSuccess ||
             cudaFuncSetAttribute(nvfp4::nvfp4_gemv_a16_kernel<2>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 nvfp4::GemvLayout<2>::kBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(nvfp4::nvfp4_gemv_a16_kernel<4>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 nvfp4::GemvLayout<4>::kBytes) != cudaSuccess)
+                                 nvfp4::GemvLayout<2>::kBytes) != cudaSuccess)
             return;
         for (int c = 2; c <= 8; ++c) {
             cudaLaunchConfig_t cfg = {};
@@ -653,9 +650,12 @@ fp8bq_status fp8bq_nvfp4_gemm_a16(const void *x_bf16, const uint8_t *packed, con
     const int64_t mtiles = (M + nvfp4::MT - 1) / nvfp4::MT;
     if (mtiles > 65535) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
     CUtensorMap tw, ts, tx;
-    if (M <= 4) {
-        // a handful of tokens: packed codes decoded in registers on the CUDA cores
-        const int MB = M <= 1 ? 1 : M <= 2 ? 2 : 4;
+    if (M <= 2) {
+        // one or two tokens: packed codes decoded in registers on the CUDA cores
+        // (from M = 3 on the tensor-core kernel, whose time hardly depends on M
+        // up to its 16-row tile, is faster: at M = 4 the CUDA-core kernel took
+        // 37.9 us against 28.9 us on fused QKV [9216, 7168])
+        const int MB = M <= 1 ? 1 : 2;
         if (!make_tmap_2d(&tw, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tmap_2d(&ts, sb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 16, 16, 128,
@@ -674,13 +674,9 @@ fp8bq_status fp8bq_nvfp4_gemm_a16(const void *x_bf16, const uint8_t *packed, con
             e = launch_clustered(nvfp4::nvfp4_gemv_a16_kernel<1>, grid, block,
                                  nvfp4::GemvLayout<1>::kBytes, st, cl, tw, ts, tx, g, yp, iM, iN, iK,
                                  iS, d->status);
-        else if (MB == 2)
+        else
             e = launch_clustered(nvfp4::nvfp4_gemv_a16_kernel<2>, grid, block,
                                  nvfp4::GemvLayout<2>::kBytes, st, cl, tw, ts, tx, g, yp, iM, iN, iK,
-                                 iS, d->status);
-        else
-            e = launch_clustered(nvfp4::nvfp4_gemv_a16_kernel<4>, grid, block,
-                                 nvfp4::GemvLayout<4>::kBytes, st, cl, tw, ts, tx, g, yp, iM, iN, iK,
                                  iS, d->status);
         return from_cuda(e);
     }

@@ -399,7 +399,7 @@ nvfp4_gemm_a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
 }
 
 
-// ---------------------------------------------------------------- GEMV (M <= 4)
+// ---------------------------------------------------------------- GEMV (M <= 2)
 //
 // For a handful of tokens the tensor-core path above is bound by shared-memory
 // traffic (a 4 KB BF16 tile per 512 codes, written and read again).  This
@@ -437,7 +437,7 @@ nvfp4_gemv_a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_x, const float *__restrict__ g_ptr,
                       __nv_bfloat16 *__restrict__ y, int M, int N, int K, int cluster_s,
                       int *status) {
-    static_assert(MB == 1 || MB == 2 || MB == 4, "token count bucket");
+    static_assert(MB == 1 || MB == 2, "token count bucket");
     using L = GemvLayout<MB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
