@@ -56,6 +56,8 @@ class Fp8bqError(RuntimeError):
 def lib() -> ctypes.CDLL:
     """Loads libfp8bq.so (raises if it has not been built)."""
     global _lib
+    if _lib is not None:  # loaded: no lock on the per-call path
+        return _lib
     with _lock:
         if _lib is not None:
             return _lib
@@ -85,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_launch_count.restype = ctypes.c_uint64
         L.fp8bq_version.argtypes = []
         L.fp8bq_version.restype = ctypes.c_int
+        L.fp8bq_clear_cache.argtypes = []
+        L.fp8bq_clear_cache.restype = None
         for name in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
                      "fp8bq_workspace_init", "fp8bq_last_device_status", "fp8bq_gemm_noalloc",
                      "fp8bq_selftest_timeout", "fp8bq_kv_write_e4m3", "fp8bq_silu_mul_quantize",
@@ -103,7 +107,13 @@ def _check(status: int, what: str) -> None:
         raise Fp8bqError(status, what)
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(t: torch.Tensor) -> ctypes.c_void_p:
+    # the current stream's handle without building a torch.cuda.Stream object
+    if _raw_stream is not None:
+        return ctypes.c_void_p(_raw_stream(t.device.index))
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
@@ -231,6 +241,11 @@ def selftest_timeout(limit_us: int = 20000) -> None:
     _check(lib().fp8bq_selftest_timeout(limit_us,
                                         ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)),
            "fp8bq_selftest_timeout")
+
+
+def clear_cache() -> None:
+    """Empties the library's cache of encoded TMA descriptors."""
+    lib().fp8bq_clear_cache()
 
 
 def launch_count() -> int:

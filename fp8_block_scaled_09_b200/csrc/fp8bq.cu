@@ -27,6 +27,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 #include <utility>
 
 #include "fp8bq.h"
@@ -286,13 +287,52 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     return launch_clustered(kernel, grid, block, smem, st, 1u, std::forward<Args>(args)...);
 }
 
-// 2-D uint8 tensor map over a row-major [rows, cols] byte matrix, box
-// [box_rows, 128 bytes], 128-byte swizzle, zero fill out of bounds.
+// Encoded tensor maps, keyed on everything the encoding depends on (address,
+// shape, element type, box and swizzle): an entry is valid for any tensor that
+// matches its key, whatever that memory held before, so entries never go stale.
+// Bounded; fp8bq_clear_cache() empties it.
+struct TmapKey {
+    uintptr_t ptr;
+    int64_t rows, cols;
+    uint32_t box_cols, box_rows;
+    int type, elem_bytes, swizzle;
+    bool operator==(const TmapKey &o) const {
+        return ptr == o.ptr && rows == o.rows && cols == o.cols && box_cols == o.box_cols &&
+               box_rows == o.box_rows && type == o.type && elem_bytes == o.elem_bytes &&
+               swizzle == o.swizzle;
+    }
+};
+struct TmapKeyHash {
+    size_t operator()(const TmapKey &k) const {
+        uint64_t h = static_cast<uint64_t>(k.ptr) * 0x9E3779B97F4A7C15ull;
+        const uint64_t parts[5] = {static_cast<uint64_t>(k.rows), static_cast<uint64_t>(k.cols),
+                                   (static_cast<uint64_t>(k.box_cols) << 32) | k.box_rows,
+                                   (static_cast<uint64_t>(k.type) << 16) |
+                                       static_cast<uint64_t>(k.elem_bytes),
+                                   static_cast<uint64_t>(k.swizzle)};
+        for (uint64_t p : parts) h = (h ^ p) * 0x100000001B3ull;
+        return static_cast<size_t>(h ^ (h >> 29));
+    }
+};
+constexpr size_t kTmapCacheMax = 4096;
+std::mutex g_tmap_mu;
+std::unordered_map<TmapKey, CUtensorMap, TmapKeyHash> g_tmap_cache;
+
 // 2-D tensor map over a row-major [rows, cols] matrix of `type` (elem_bytes each),
 // box [box_rows, box_cols], zero fill out of bounds.
 bool make_tmap_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType type, int elem_bytes,
                   int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows,
                   CUtensorMapSwizzle swizzle) {
+    const TmapKey key{reinterpret_cast<uintptr_t>(ptr), rows, cols, box_cols, box_rows,
+                      static_cast<int>(type), elem_bytes, static_cast<int>(swizzle)};
+    {
+        std::lock_guard<std::mutex> lk(g_tmap_mu);
+        auto it = g_tmap_cache.find(key);
+        if (it != g_tmap_cache.end()) {
+            *map = it->second;
+            return true;
+        }
+    }
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -300,23 +340,21 @@ bool make_tmap_2d(CUtensorMap *map, const void *ptr, CUtensorMapDataType type, i
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t elem[2] = {1u, 1u};
     std::memset(map, 0, sizeof(*map));
-    return enc(map, type, 2, const_cast<void *>(ptr), dims, strides, box, elem,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (enc(map, type, 2, const_cast<void *>(ptr), dims, strides, box, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lk(g_tmap_mu);
+    if (g_tmap_cache.size() >= kTmapCacheMax) g_tmap_cache.clear();
+    g_tmap_cache.emplace(key, *map);
+    return true;
 }
 
+// 2-D uint8 tensor map over a row-major [rows, cols] byte matrix, box
+// [box_rows, 128 bytes], 128-byte swizzle, zero fill out of bounds.
 bool make_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, uint32_t box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
-    const cuuint32_t box[2] = {128u, box_rows};
-    const cuuint32_t elem[2] = {1u, 1u};
-    std::memset(map, 0, sizeof(*map));
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box,
-               elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return make_tmap_2d(map, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, cols, 128u, box_rows,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 size_t round256(int64_t b) { return static_cast<size_t>(((b + 255) / 256) * 256); }
@@ -785,6 +823,11 @@ const char *fp8bq_status_string(fp8bq_status status) {
 uint64_t fp8bq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int fp8bq_version(void) { return 100; }
+
+void fp8bq_clear_cache(void) {
+    std::lock_guard<std::mutex> lk(g_tmap_mu);
+    g_tmap_cache.clear();
+}
 
 fp8bq_status fp8bq_selftest_timeout(uint32_t limit_us, void *stream) {
     if (limit_us == 0 || limit_us > 2000000u) return FP8BQ_ERR_INVALID_ARG;

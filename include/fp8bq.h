@@ -270,6 +270,13 @@ FP8BQ_API uint64_t fp8bq_launch_count(void);
 /* ABI version: major * 10000 + minor * 100 + patch. */
 FP8BQ_API int fp8bq_version(void);
 
+/* The library keeps the TMA descriptors it encodes, keyed on everything an
+ * encoding depends on (address, shape, element type, box, swizzle), so a
+ * repeated call skips the encoding; an entry is valid for any tensor matching
+ * its key, so entries never go stale.  The cache is bounded (it empties itself
+ * when full); this call empties it now.  Host memory only; thread-safe. */
+FP8BQ_API void fp8bq_clear_cache(void);
+
 #ifdef __cplusplus
 }
 #endif

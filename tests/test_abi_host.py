@@ -201,6 +201,12 @@ def test_valid_call_without_device_reports_no_device(L):
     assert L.fp8bq_nvfp4_gemm_a16(GOOD, GOOD, GOOD, GOOD, 4, 128, 256, GOOD, None) == NODEV
 
 
+def test_descriptor_cache_clears_without_a_device(L):
+    # host-only: the cache of encoded TMA descriptors needs no GPU to be emptied
+    fp8bq.clear_cache()
+    fp8bq.clear_cache()
+
+
 def test_selftest_limit_is_validated_on_the_host(L):
     assert L.fp8bq_selftest_timeout(0, None) == INVALID
     assert L.fp8bq_selftest_timeout(2000001, None) == INVALID

@@ -191,6 +191,31 @@ def test_linear_matches_oracle_and_unfused_path(M, N, K):
     assert torch.equal(y.t.view(torch.int16), y2.view(torch.int16))
 
 
+# ------------------------------------------------------------------ descriptor cache
+
+@pytest.mark.parametrize("M,N,K", [(8, 1024, 1024), (300, 512, 1024)])
+def test_descriptor_cache_reuse_new_contents_and_clear(M, N, K):
+    # Repeated calls on the same buffers reuse the cached TMA descriptors; a
+    # descriptor names an address, not contents, so new data in the same
+    # buffers must be read; clearing the cache changes nothing either.
+    dev = [torch.empty((M, K), dtype=torch.uint8, device="cuda"),
+           torch.empty((M, K // 128), dtype=torch.float32, device="cuda"),
+           torch.empty((N, K), dtype=torch.uint8, device="cuda"),
+           torch.empty((N // 128, K // 128), dtype=torch.float32, device="cuda")]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = fp8bq.new_workspace(fp8bq.OP_GEMM, M, N, K, "cuda")
+    for i, clear in enumerate((False, False, True)):
+        x, qa, sa, qw, sw = operands(M, N, K, 940 + 7 * i)
+        for d, h in zip(dev, (qa, sa, qw, sw)):
+            d.copy_(torch.from_numpy(np.ascontiguousarray(
+                h, dtype=np.float32 if d.dtype == torch.float32 else np.uint8)))
+        if clear:
+            fp8bq.clear_cache()
+        fp8bq.gemm(*dev, out=y, workspace=ws)
+        torch.cuda.synchronize()
+        check(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
+
+
 # ------------------------------------------------------------------ stream order
 
 def test_weights_quantized_right_before_the_linear():
