@@ -53,7 +53,7 @@ ROTATE = 4                   # device copies of each decode weight
 # DRAM bytes (read + write) of one decode GEMM launch, o_proj M=1 (7168 x 7168), from the ncu
 # capture summarised in profiles/gemm_decode_kernel_o_proj_m1.md; scaled to other shapes by
 # their algorithmic bytes (the capture shows DRAM bytes = algorithmic bytes within 0.04%).
-DECODE_TRAFFIC_CAPTURE = {"shape": (1, 7168, 7168), "dram_bytes": 51_472_640 + 28_928,
+DECODE_TRAFFIC_CAPTURE = {"shape": (1, 7168, 7168), "dram_bytes": 51_472_896 + 5_888,
                           "source": "profiles/gemm_decode_kernel_o_proj_m1.md"}
 DECODE_WORKLOAD = ("decode GEMV set: fp8bq_linear, M in {1,4,8} x {fused QKV W[9216,7168], "
                    "o_proj W[7168,7168]}, E4M3 128x128-blocked weights, X BF16 N(0,1) with "
