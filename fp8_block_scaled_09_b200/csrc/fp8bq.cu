@@ -3,7 +3,9 @@
 //
 // All kernels live in this one translation unit so the device status word is a
 // single per-device symbol.  Dispatch:
-//   quantize_act     -> quantize_act_kernel (HBM-bound, persistent, bulk-copy ring)
+//   quantize_act     -> up to 8192 groups: quantize_act_small_kernel (no shared
+//                       memory, fits beside a running GEMM); larger:
+//                       quantize_act_kernel (HBM-bound, persistent, bulk-copy ring)
 //   quantize_weight  -> quantize_weight_kernel (one CTA per 128x128 block)
 //   gemm, M <= 128   -> decode::gemm_decode_kernel<MT> (token tile MT = 16, 32,
 //                       64 or 128; each n-block split over a cluster of CTAs
