@@ -27,6 +27,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
@@ -70,8 +71,12 @@ constexpr int kPrefillBN = 256;
 // The CTA-pair prefill kernel is correct and, moving 2/3 of the operand bytes,
 // runs exactly as fast as the single-CTA kernel (both are bound by the
 // per-chunk TMEM hand-off, not by L2), and no faster under the power cap; the
-// single-CTA kernel stays the one dispatched.
-constexpr bool kUsePairPrefill = false;
+// single-CTA kernel is the one dispatched unless the environment variable
+// FP8BQ_PREFILL_PAIRS=1 selects the pair kernel (read once per device).
+bool pair_prefill_requested() {
+    const char *v = std::getenv("FP8BQ_PREFILL_PAIRS");
+    return v != nullptr && v[0] == '1' && v[1] == '\0';
+}
 constexpr int64_t kDecodeMaxM = decode::kMaxMT;
 
 std::atomic<uint64_t> g_launches{0};
@@ -137,7 +142,7 @@ const DeviceInfo *device_info() {
             return;
         // CTA-pair prefill kernel: optional; any failure here only leaves it off.
         d.pair_clusters = 0;
-        if (kUsePairPrefill &&
+        if (pair_prefill_requested() &&
             cudaFuncSetAttribute(prefill2::gemm_prefill_pair_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  prefill2::Layout::kDynamicSmem) == cudaSuccess &&
@@ -512,7 +517,7 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
             default:
                 return launch_decode<128>(d, qa, sa, qw, sw, M, N, K, y, ws, st, err, early_weights, plan);
         }
-    } else if (kUsePairPrefill && d.pair_clusters > 0 && M > prefill::BM) {
+    } else if (d.pair_clusters > 0 && M > prefill::BM) {
         // CTA pairs: each CTA loads 128 rows of A and 128 of the 256 weight rows
         CUtensorMap ta, tb;
         if (!make_tmap(&ta, qa, M, K, prefill2::kHalf) || !make_tmap(&tb, qw, N, K, prefill2::kHalf)) {

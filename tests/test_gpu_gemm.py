@@ -11,6 +11,10 @@ workload shapes are checked on sampled rows.  In the exact-arithmetic regime
 (small-integer codes, power-of-two scales) every partial sum is exact in FP32,
 so the output must equal the BF16 rounding of the exact result bit for bit.
 """
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -189,6 +193,49 @@ def test_linear_matches_oracle_and_unfused_path(M, N, K):
     gq, gs = fp8bq.quantize_act(xd)
     y2 = fp8bq.gemm(gq, gs, to_dev_codes(qw), to_dev_f32(sw))
     assert torch.equal(y.t.view(torch.int16), y2.view(torch.int16))
+
+
+# ------------------------------------------------------------------ CTA-pair prefill kernel
+
+_PAIR_CHECK = r"""
+import numpy as np, torch
+import fp8_block_scaled_09_b200 as fp8bq, oracle, workloads
+from gpu_util import bf16_to_f64, to_dev_codes, to_dev_f32, tolerance_report
+for i, (M, N, K) in enumerate([(300, 512, 1024), (1000, 768, 2048), (256, 1152, 7168),
+                               (129, 256, 256)]):
+    x = workloads.activation(M, K, 960 + i, outliers=2)
+    qa, sa = oracle.quantize_act(x)
+    qw, sw = oracle.quantize_weight(workloads.weight(N, K, 970 + i))
+    y = fp8bq.gemm(to_dev_codes(qa), to_dev_f32(sa), to_dev_codes(qw), to_dev_f32(sw))
+    torch.cuda.synchronize()
+    ok, ratio, _ = tolerance_report(bf16_to_f64(y), oracle.gemm_ref(qa, sa, qw, sw))
+    assert ok, (M, N, K, ratio)
+rng = np.random.default_rng(5)
+small = np.array([0x00, 0x38, 0x40, 0x44, 0xB8, 0xC0], np.uint8)
+M, N, K = 384, 512, 1024
+qa, qw = rng.choice(small, size=(M, K)), rng.choice(small, size=(N, K))
+sa = np.ldexp(np.float32(1.0), rng.integers(-2, 3, size=(M, K // 128))).astype(np.float32)
+sw = np.ldexp(np.float32(1.0), rng.integers(-2, 3, size=(N // 128, K // 128))).astype(np.float32)
+y = fp8bq.gemm(to_dev_codes(qa), to_dev_f32(sa), to_dev_codes(qw), to_dev_f32(sw))
+torch.cuda.synchronize()
+exp = oracle.bf16_round(oracle.gemm_ref(qa, sa, qw, sw))  # BF16 bit patterns
+assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16), exp)
+assert fp8bq.last_device_status() == 0
+print("pair prefill ok")
+"""
+
+
+def test_pair_prefill_kernel_when_selected():
+    # The CTA-pair prefill kernel is off by default; FP8BQ_PREFILL_PAIRS=1 (read
+    # once per device) selects it, so it runs in a process of its own.
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    env = dict(os.environ, FP8BQ_PREFILL_PAIRS="1",
+               PYTHONPATH=os.pathsep.join([root, here, os.environ.get("PYTHONPATH", "")]))
+    r = subprocess.run([sys.executable, "-c", _PAIR_CHECK], env=env, capture_output=True,
+                       text=True, timeout=900, cwd=root)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
+    assert "pair prefill ok" in r.stdout
 
 
 # ------------------------------------------------------------------ descriptor cache
