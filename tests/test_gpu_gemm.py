@@ -63,11 +63,12 @@ def check(y, ref):
 
 # Up to 148 n-blocks the decode kernel splits each n-block over a cluster of
 # CTAs (sizes 1-8: e.g. 2 for QKV, 3 for (2, 256, 384), 5 for (7, 640, 640), 8
-# for k_proj); beyond that it runs stream-K with the global split-K reduction
-# ((4, 19200, 512), (3, 32768, 256)).
+# for k_proj, (9, 2048, 2048) and (5, 1280, 1536)); beyond that it runs
+# stream-K with the global split-K reduction ((4, 19200, 512), (3, 32768, 256)).
 DECODE_SHAPES = [(1, 128, 128), (1, 1024, 7168), (2, 256, 384), (4, 9216, 7168),
                  (8, 7168, 7168), (15, 384, 1024), (16, 1024, 7168), (16, 128, 21504),
-                 (3, 16384, 256), (7, 640, 640), (4, 19200, 512), (3, 32768, 256)]
+                 (3, 16384, 256), (7, 640, 640), (4, 19200, 512), (3, 32768, 256),
+                 (9, 2048, 2048), (5, 1280, 1536)]
 
 
 @pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
