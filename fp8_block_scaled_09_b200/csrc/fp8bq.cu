@@ -438,12 +438,27 @@ DecodePlan decode_plan(const DeviceInfo &d, int64_t M, int64_t N, int64_t K) {
     return p;
 }
 
+// Workspace the GEMM requires: the decode path's, whenever that path may be
+// chosen (the choice needs the device's SM count; the size does not).
 size_t gemm_ws_bytes(int64_t M, int64_t N) {
-    // sized for the decode path whenever it may be chosen (the choice needs the
-    // device's SM count; the workspace does not depend on it)
     if (M <= kDecodeMaxM && N / 128 <= decode::kMaxCounters)
         return round256(decode::workspace_bytes(N / 128, decode::token_tile(M)));
     return 0;
+}
+
+// Prefill split-K tail: the counter header, then kTailMaxTiles x kTailMaxParts
+// FP32 partial tiles.  Optional: a smaller workspace runs without the split.
+constexpr size_t kPrefillTailBytes =
+    size_t(decode::kCounterBytes) +
+    size_t(prefill::kTailMaxTiles) * prefill::kTailMaxParts * prefill::kTailPartialFloats * 4;
+
+constexpr int64_t kPrefillTailMinKB = 128;  // K >= 16384
+
+// Workspace fp8bq_workspace_size reports: what the GEMM requires, or for the
+// prefill path what its split-K tail can use.
+size_t gemm_ws_bytes_full(int64_t M, int64_t N) {
+    const size_t need = gemm_ws_bytes(M, N);
+    return M > kDecodeMaxM ? std::max(need, round256(kPrefillTailBytes)) : need;
 }
 
 size_t act_ws_bytes(int64_t M, int64_t K) { return round256(M * K) + round256(M * (K / 128) * 4); }
@@ -500,9 +515,11 @@ cudaError_t launch_decode(const DeviceInfo &d, const uint8_t *qa, const float *s
 // its dependency wait (only valid right after this library's activation
 // quantizer, while the GEMM before it may still be running; see
 // gemm_decode.cuh).
+// ws_bytes: usable workspace bytes (the prefill path splits its last wave of
+// tiles K-wise when they hold kPrefillTailBytes).
 cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
                         const uint8_t *qw, const float *sw, int64_t M, int64_t N, int64_t K,
-                        void *y, void *ws, cudaStream_t st, fp8bq_status *err,
+                        void *y, void *ws, size_t ws_bytes, cudaStream_t st, fp8bq_status *err,
                         bool early_weights = false, bool allow_decode = true) {
     *err = FP8BQ_OK;
     const DecodePlan plan = decode_plan(d, M, N, K);
@@ -539,10 +556,26 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
         }
         const int64_t tiles = ((M + prefill::BM - 1) / prefill::BM) * ((N + kPrefillBN - 1) / kPrefillBN);
         const int grid = static_cast<int>(tiles < d.sm_count ? tiles : d.sm_count);
+        // A last wave of at most kTailMaxTiles tiles leaves most SMs idle: split
+        // each of its tiles K-wise into up to kTailMaxParts parts.  Measured: it
+        // pays for long K (M=4096, N=7168: K=21504 681 -> 631 us) but not for
+        // K=8192 (269 -> 278 us), where the partial hand-off outweighs it.
+        const int64_t KB = K / 128, rest = tiles % grid;
+        int tail_parts = 0;
+        if (ws != nullptr && aligned16(ws) && ws_bytes >= kPrefillTailBytes && tiles > grid && rest >= 1 &&
+            rest <= prefill::kTailMaxTiles && KB >= kPrefillTailMinKB)
+            tail_parts = static_cast<int>(std::min<int64_t>(
+                std::min<int64_t>(prefill::kTailMaxParts, grid / rest), KB));
+        if (tail_parts < 2) tail_parts = 0;
+        int *tail_counters = tail_parts ? static_cast<int *>(ws) : nullptr;
+        float *tail_partials =
+            tail_parts ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes)
+                       : nullptr;
         return launch(prefill::gemm_prefill_kernel<kPrefillBN>, dim3(grid),
                       dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN>::kDynamicSmem, st,
                       ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
-                      static_cast<int>(N), static_cast<int>(K), d.status);
+                      static_cast<int>(N), static_cast<int>(K), d.status, tail_parts, tail_partials,
+                      tail_counters);
     }
 }
 
@@ -741,8 +774,8 @@ fp8bq_status fp8bq_nvfp4_gemm_a16(const void *x_bf16, const uint8_t *packed, con
 
 size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {
     if (check_mnk(M, N, K) != FP8BQ_OK || M == 0) return 0;
-    if (op == FP8BQ_OP_GEMM) return gemm_ws_bytes(M, N);
-    if (op == FP8BQ_OP_LINEAR) return act_ws_bytes(M, K) + gemm_ws_bytes(M, N);
+    if (op == FP8BQ_OP_GEMM) return gemm_ws_bytes_full(M, N);
+    if (op == FP8BQ_OP_LINEAR) return act_ws_bytes(M, K) + gemm_ws_bytes_full(M, N);
     return 0;
 }
 
@@ -762,7 +795,7 @@ fp8bq_status fp8bq_gemm(const uint8_t *qa, const float *sa, const uint8_t *qw, c
     if (!d) return FP8BQ_ERR_NO_DEVICE;
     fp8bq_status err;
     cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, workspace,
-                                static_cast<cudaStream_t>(stream), &err);
+                                workspace ? ws_bytes : 0, static_cast<cudaStream_t>(stream), &err);
     if (err != FP8BQ_OK) return err;
     return from_cuda(e);
 }
@@ -789,7 +822,8 @@ fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const float *sw
     cudaError_t e = launch_quantize_act(*d, x_bf16, M, K, qa, sa, s);
     if (e != cudaSuccess) return FP8BQ_ERR_CUDA;
     fp8bq_status err;
-    e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, gemm_ws, s, &err, /*early_weights=*/true);
+    e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, gemm_ws, ws_bytes - act_ws_bytes(M, K), s,
+                    &err, /*early_weights=*/true);
     if (err != FP8BQ_OK) return err;
     return from_cuda(e);
 }
@@ -878,7 +912,8 @@ fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, const uint8_
                                 s) != cudaSuccess)
         return FP8BQ_ERR_CUDA;
     fp8bq_status err;
-    cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, g_noalloc_ptr[dev], s, &err,
+    cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, g_noalloc_ptr[dev],
+                                /*ws_bytes (no prefill tail split)=*/0, s, &err,
                                 /*early_weights=*/false, /*allow_decode=*/fits);
     if (err != FP8BQ_OK) return err;
     return from_cuda(e);

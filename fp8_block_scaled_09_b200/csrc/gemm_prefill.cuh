@@ -68,6 +68,37 @@ struct Layout {
     static constexpr uint32_t kTmemCols = 2 * BN;
 };
 
+// Split-K tail: when the tiles leave a last wave of at most kTailMaxTiles tiles
+// on the persistent grid, each of those tiles is split K-wise into tail_parts
+// parts run by different CTAs; each part's FP32 partial goes to the workspace
+// and the part that finishes last sums all of them in part order
+// (deterministic) and writes the tile.
+constexpr int kTailMaxTiles = 16;
+constexpr int kTailMaxParts = 4;
+constexpr int64_t kTailPartialFloats = int64_t(BM) * 256;  // one part of a 128 x 256 tile
+
+// The CTA's w-th work item: first its full tiles (blockIdx.x + w gridDim.x
+// below full_tiles), then at most one tail part.  part < 0 for a full tile.
+__device__ __forceinline__ bool work_item(int w, int num_tiles, int full_tiles, int tail_parts,
+                                          int KB, int &tile, int &kb0, int &kb1, int &part) {
+    const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    const int t = c + w * G;
+    if (t < full_tiles) {
+        tile = t;
+        kb0 = 0;
+        kb1 = KB;
+        part = -1;
+        return true;
+    }
+    if (tail_parts == 0 || w != (full_tiles - c + G - 1) / G) return false;
+    if (c >= (num_tiles - full_tiles) * tail_parts) return false;
+    tile = full_tiles + c / tail_parts;
+    part = c % tail_parts;
+    kb0 = part * KB / tail_parts;
+    kb1 = (part + 1) * KB / tail_parts;
+    return true;
+}
+
 __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int &tm, int &tn) {
     const int group = kGroupM * n_tiles;
     const int g = t / group, r = t - g * group;
@@ -233,7 +264,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const float *__restrict__ sa,
                     const float *__restrict__ sw, __nv_bfloat16 *__restrict__ y, int M, int N,
-                    int K, int *status) {
+                    int K, int *status, int tail_parts, float *tail_partials, int *tail_counters) {
     using L = Layout<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -251,6 +282,9 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const int m_tiles = (M + BM - 1) / BM;
     const int n_tiles = (N + BN - 1) / BN;
     const int num_tiles = m_tiles * n_tiles;
+    // with a split-K tail, the last wave's tiles are split into parts
+    const int full_tiles =
+        tail_parts > 0 ? num_tiles - num_tiles % static_cast<int>(gridDim.x) : num_tiles;
 
     allow_dependent_launch();
     if (threadIdx.x == 0) {
@@ -264,6 +298,8 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
         mbar_init(drain, 2);
         *abort_flag = 0;
+        reinterpret_cast<uint32_t *>(smem + L::kMiscOff + 8)[0] = 0;  // tail verdict
+        reinterpret_cast<uint32_t *>(smem + L::kMiscOff + 8)[1] = 0;  // tail arrivals
         fence_barrier_init();
         prefetch_tmap(&tmap_a);
         prefetch_tmap(&tmap_b);
@@ -288,10 +324,12 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 uint32_t stage = 0, phase = 0;
                 int64_t issued = 0;
                 bool ok = true;
-                for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                int t, kb0, kb1, part;
+                for (int w = 0; ok && work_item(w, num_tiles, full_tiles, tail_parts, KB, t, kb0, kb1, part);
+                     ++w) {
                     int tm, tn;
                     tile_coords(t, m_tiles, n_tiles, tm, tn);
-                    for (int kb = 0; kb < KB; ++kb) {
+                    for (int kb = kb0; kb < kb1; ++kb) {
                         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) {
                             ok = false;
                             break;
@@ -321,8 +359,10 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const uint32_t buf = static_cast<uint32_t>(warp - 1);
                 int64_t i = 0;
                 bool ok = true;
-                for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                    for (int kb = 0; kb < KB; ++kb, ++i) {
+                int t, kb0, kb1, part;
+                for (int w = 0; ok && work_item(w, num_tiles, full_tiles, tail_parts, KB, t, kb0, kb1, part);
+                     ++w) {
+                    for (int kb = kb0; kb < kb1; ++kb, ++i) {
                         if ((i & 1) != buf) continue;
                         const uint32_t stage = static_cast<uint32_t>(i % kStages);
                         const uint32_t phase = static_cast<uint32_t>((i / kStages) & 1);
@@ -356,9 +396,15 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int quarter = warp & 3;  // TMEM lane quarter accessible to this warp
         const int half = pw >> 2;      // which 128-column weight block of the tile
         const int row_in_tile = quarter * 32 + lane;
+        const int pt = threadIdx.x - kFirstPromoWarp * 32;  // 0..255
+        // tail part hand-shake: arrivals of the promotion warps, then the verdict
+        volatile uint32_t *tail_last = reinterpret_cast<volatile uint32_t *>(smem + L::kMiscOff + 8);
+        uint32_t *tail_arrived = reinterpret_cast<uint32_t *>(smem + L::kMiscOff + 12);
         uint32_t buf = 0, bphase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int t, kb0, kb1, part;
+        for (int w = 0; ok && work_item(w, num_tiles, full_tiles, tail_parts, KB, t, kb0, kb1, part);
+             ++w) {
             int tm, tn;
             tile_coords(t, m_tiles, n_tiles, tm, tn);
             const int grow = tm * BM + row_in_tile;
@@ -375,17 +421,17 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             float sa_q[kScaleLookahead], sw_q[kScaleLookahead];
 #pragma unroll
             for (int j = 0; j < kScaleLookahead; ++j) {
-                sa_q[j] = (row_ok && j < KB) ? __ldg(sa_row + j) : 0.0f;
-                sw_q[j] = (col_ok && j < KB) ? __ldg(sw_row + j) : 0.0f;
+                sa_q[j] = (row_ok && kb0 + j < kb1) ? __ldg(sa_row + kb0 + j) : 0.0f;
+                sw_q[j] = (col_ok && kb0 + j < kb1) ? __ldg(sw_row + kb0 + j) : 0.0f;
             }
-            for (int kb0 = 0; kb0 < KB && ok; kb0 += kScaleLookahead) {
+            for (int kbb = kb0; kbb < kb1 && ok; kbb += kScaleLookahead) {
 #pragma unroll
                 for (int j = 0; j < kScaleLookahead; ++j) {
-                    const int kb = kb0 + j;
-                    if (kb >= KB) break;
+                    const int kb = kbb + j;
+                    if (kb >= kb1) break;
                     const float scale = sa_q[j] * sw_q[j];
                     const int kn = kb + kScaleLookahead;
-                    if (kn < KB) {
+                    if (kn < kb1) {
                         sa_q[j] = row_ok ? __ldg(sa_row + kn) : 0.0f;
                         sw_q[j] = col_ok ? __ldg(sw_row + kn) : 0.0f;
                     }
@@ -408,7 +454,59 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     if (buf == 0) bphase ^= 1;
                 }
             }
-            if (ok && row_ok && col_ok) {
+            if (!ok) break;
+            const bool write = part < 0;  // full tile: write its output from registers
+            if (part >= 0) {
+                // Tail part: publish the FP32 partial [128 rows][256 cols] of
+                // this part; the part that arrives last sums them all.
+                const int r = t - full_tiles;
+                const int64_t unit = static_cast<int64_t>(r) * tail_parts + part;
+                float4 *dst = reinterpret_cast<float4 *>(tail_partials + unit * kTailPartialFloats +
+                                                         row_in_tile * 256 + half * 128);
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    __stcg(dst + c, make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]));
+                // Every promotion warp's stores are published, then one thread
+                // takes the tile's counter: 2 in *tail_last if this part is the
+                // last to arrive, 1 otherwise.  (Flags in shared memory with
+                // the usual bounded waits, so an abandoned wait elsewhere can
+                // never leave a warp stuck here.)
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(tail_arrived, 1u);
+                if (pt == 0) {
+                    if (smem_flag_wait(tail_arrived, static_cast<uint32_t>(kPromoWarps), abort_flag, status))
+                        *tail_last = atomicAdd(&tail_counters[r], 1) == tail_parts - 1 ? 2u : 1u;
+                }
+                if (!smem_flag_wait(tail_last, 1u, abort_flag, status)) break;
+                if (*tail_last == 2u && row_ok && col_ok) {
+                    // Last part: sum every part's partial (this one's included,
+                    // re-read from L2) in part order and write the tile's BF16
+                    // output, four columns at a time.
+                    __threadfence();
+                    const float4 *base = reinterpret_cast<const float4 *>(
+                        tail_partials + static_cast<int64_t>(r) * tail_parts * kTailPartialFloats +
+                        row_in_tile * 256 + half * 128);
+                    uint2 *yrow = reinterpret_cast<uint2 *>(y + static_cast<int64_t>(grow) * N + gcol);
+                    // (eight column groups at a time, so their loads overlap)
+#pragma unroll 8
+                    for (int c = 0; c < 32; ++c) {
+                        float4 s4 = __ldcg(base + c);
+#pragma unroll
+                        for (int pp = 1; pp < kTailMaxParts; ++pp) {
+                            if (pp >= tail_parts) break;
+                            const float4 v = __ldcg(base + pp * (kTailPartialFloats / 4) + c);
+                            s4.x += v.x;
+                            s4.y += v.y;
+                            s4.z += v.z;
+                            s4.w += v.w;
+                        }
+                        yrow[c] = make_uint2(pack_bf16x2(s4.x, s4.y), pack_bf16x2(s4.z, s4.w));
+                    }
+                }
+                if (*tail_last == 2u && pt == 0) tail_counters[r] = 0;  // zeroed for the next call
+            }
+            if (write && row_ok && col_ok) {
                 uint4 *dst = reinterpret_cast<uint4 *>(y + static_cast<int64_t>(grow) * N + gcol);
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {

@@ -96,6 +96,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Waits (bounded, like mbar_wait) until the shared-memory word *flag is at
+// least `target`.
+__device__ __forceinline__ bool smem_flag_wait(const volatile uint32_t *flag, uint32_t target,
+                                               volatile int *abort, int *status,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+    if (*flag >= target) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (*flag >= target) return true;
+        if ((it & 255u) == 0) {
+            if (abort != nullptr && *abort) return false;
+            if (global_timer_ns() - t0 > limit_ns) {
+                if (abort != nullptr) *abort = 1;
+                atomicExch(status, 6 /* FP8BQ_ERR_TIMEOUT */);
+                return false;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {

@@ -112,7 +112,7 @@ FP8BQ_API fp8bq_status fp8bq_quantize_weight(const void *w_bf16, int64_t N, int6
  *   y_bf16 : out, BF16 [M, N]
  *   workspace, ws_bytes : device scratch of at least
  *       fp8bq_workspace_size(FP8BQ_OP_GEMM, M, N, K) bytes (may be NULL when
- *       that is 0).  Its contents must be the state left by
+ *       that is 0; for M > 128 optional, see fp8bq_workspace_size).  Its contents must be the state left by
  *       fp8bq_workspace_init() or by any previous successful fp8bq_gemm or
  *       fp8bq_linear call, of any shape (every successful call restores that
  *       state); calls that share a workspace must be ordered (same stream).
@@ -240,8 +240,13 @@ FP8BQ_API fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, co
                                           const float *sw, int64_t M, int64_t N, int64_t K,
                                           void *y_bf16, void *stream);
 
-/* Bytes of workspace the operation needs for this shape (0 when none, and for
- * arguments the call would reject).  Always a multiple of 256. */
+/* Bytes of workspace the operation uses for this shape (0 when none, and for
+ * arguments the call would reject).  Always a multiple of 256.  For M <= 128
+ * the call requires at least this much.  For M > 128 (the prefill GEMM) any
+ * workspace is accepted, NULL included; with at least this much, a last wave
+ * of at most 16 output tiles on the persistent grid is split K-wise over more
+ * CTAs (FP32 partials summed in a fixed order, so results stay deterministic
+ * and within the same tolerance), which a smaller one goes without. */
 FP8BQ_API size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K);
 
 /* Put a workspace into its initial state (zero-fills ws_bytes bytes on the

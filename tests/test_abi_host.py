@@ -121,7 +121,10 @@ def test_linear_argument_errors(L):
     assert f(GOOD, GOOD, GOOD, 300, 256, 100, GOOD, GOOD, ws, None) == SHAPE
     assert f(GOOD, GOOD, None, 300, 256, 256, GOOD, GOOD, ws, None) == INVALID
     assert f(ODD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws, None) == MISALIGNED
-    assert f(GOOD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws - 256, None) == WORKSPACE
+    # for M > 128 only the activation codes and scales are required; the rest of
+    # the reported size is the prefill GEMM's optional split-K tail
+    tail = 16384 + 16 * 4 * 128 * 256 * 4
+    assert f(GOOD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws - tail - 256, None) == WORKSPACE
     assert f(None, None, None, 0, 256, 256, None, None, 0, None) == OK
 
 
@@ -173,7 +176,9 @@ def test_workspace_sizes(L):
     assert g(0, 256, 256) == 0 and lin(0, 256, 256) == 0
     assert g(8, 200, 256) == 0 and g(8, 256, 200) == 0           # rejected shapes
     assert fp8bq.workspace_size(7, 8, 256, 256) == 0              # unknown op
-    assert g(8192, 9216, 7168) == 0                              # prefill GEMM needs none
+    # prefill GEMM: optional, the split-K tail's counter header + 16 x 4 partial tiles
+    tail = 16384 + 16 * 4 * 128 * 256 * 4
+    assert g(8192, 9216, 7168) == tail
     d = g(16, 9216, 7168)
     assert d > 0 and d % 256 == 0
     # decode split-K: counters + (N/128 + 256) slots of 16 x 128 FP32 partials
@@ -182,7 +187,7 @@ def test_workspace_sizes(L):
     assert g(17, 9216, 7168) == 16384 + (72 + 256) * 32 * 128 * 4
     assert g(64, 9216, 7168) == 16384 + (72 + 256) * 64 * 128 * 4
     assert g(65, 9216, 7168) == g(128, 9216, 7168) == 16384 + (72 + 256) * 128 * 128 * 4
-    assert g(129, 9216, 7168) == 0
+    assert g(129, 9216, 7168) == tail
     # linear adds the activation codes and scales
     assert lin(8192, 9216, 7168) >= 8192 * 7168 + 8192 * 56 * 4
     assert lin(16, 9216, 7168) >= d + 16 * 7168 + 16 * 56 * 4

@@ -196,6 +196,45 @@ def test_linear_matches_oracle_and_unfused_path(M, N, K):
     assert torch.equal(y.t.view(torch.int16), y2.view(torch.int16))
 
 
+# ------------------------------------------------------------------ prefill split-K tail
+
+# (M/128) x (N/256) = 160 or 150 tiles on a 148-SM grid with K >= 16384: the
+# last wave's 12 or 2 tiles are split K-wise into parts whose FP32 partials the
+# last part sums.  (Shorter K runs without the split; (1190, 4096, 7168) checks
+# that path on the same tile count.)
+@pytest.mark.parametrize("M,N,K", [(1280, 4096, 16384), (1190, 3840, 16384), (1190, 4096, 7168)])
+def test_prefill_split_tail_matches_oracle(M, N, K):
+    x, qa, sa, qw, sw = operands(M, N, K, 980 + M + K)
+    y = run_gemm(qa, sa, qw, sw)
+    rows = sample_rows(M, 24, extra=(127, 128, 1023, 1024, 1151, 1152, M - 129))
+    check(bf16_to_f64(y)[rows], oracle.gemm_ref(qa, sa, qw, sw, rows=rows))
+
+
+def test_prefill_split_tail_exact_and_without_workspace():
+    # exact regime: the split sums are exact, so the tail split, a second call on
+    # the same workspace (its counters back at zero) and a call without the
+    # workspace (no split) all give the exact result bit for bit.  160 tiles: the
+    # last 12 in raster order (m-tiles 8, 9 of n-tile 14, all of n-tile 15) are
+    # split; rows 1024.. hold every split tile's rows.
+    M, N, K = 1280, 4096, 16384
+    rng = np.random.default_rng(77)
+    small = np.array([0x00, 0x38, 0x40, 0x44, 0xB8, 0xC0], np.uint8)
+    qa, qw = rng.choice(small, size=(M, K)), rng.choice(small, size=(N, K))
+    # scales 2^-1..2^1: every partial sum is a multiple of 2^-2 below 2^20, exact
+    sa = np.ldexp(np.float32(1.0), rng.integers(-1, 2, size=(M, K // 128))).astype(np.float32)
+    sw = np.ldexp(np.float32(1.0), rng.integers(-1, 2, size=(N // 128, K // 128))).astype(np.float32)
+    rows = np.arange(1024, M, dtype=np.int64)
+    expect = oracle.bf16_round(oracle.gemm_ref(qa, sa, qw, sw, rows=rows))  # BF16 bit patterns
+    dev = (to_dev_codes(qa), to_dev_f32(sa), to_dev_codes(qw), to_dev_f32(sw))
+    ws = fp8bq.new_workspace(fp8bq.OP_GEMM, M, N, K, "cuda")
+    assert ws.numel() > 8 << 20
+    for workspace in (ws, ws, torch.zeros(256, dtype=torch.uint8, device="cuda")):
+        y = fp8bq.gemm(*dev, workspace=workspace)
+        torch.cuda.synchronize()
+        assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16)[rows], expect)
+    assert int(ws[:64].sum()) == 0  # the tail counters are back at zero
+
+
 # ------------------------------------------------------------------ CTA-pair prefill kernel
 
 _PAIR_CHECK = r"""
