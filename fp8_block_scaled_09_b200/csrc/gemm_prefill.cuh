@@ -475,8 +475,10 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 __syncwarp();
                 if (lane == 0) atomicAdd(tail_arrived, 1u);
                 if (pt == 0) {
-                    if (smem_flag_wait(tail_arrived, static_cast<uint32_t>(kPromoWarps), abort_flag, status))
+                    if (smem_flag_wait(tail_arrived, static_cast<uint32_t>(kPromoWarps), abort_flag, status)) {
+                        __threadfence();  // the CTA's partial stores before the counter increment
                         *tail_last = atomicAdd(&tail_counters[r], 1) == tail_parts - 1 ? 2u : 1u;
+                    }
                 }
                 if (!smem_flag_wait(tail_last, 1u, abort_flag, status)) break;
                 if (*tail_last == 2u && row_ok && col_ok) {
