@@ -145,7 +145,7 @@ DRAFTER_MLP = (DRAFTER_FC, DRAFTER_GATE_UP, DRAFTER_DOWN)
 
 # workload 5: long-prefill o_proj and the standalone activation quantizer
 LONG_O_PROJ = Gemm("o_proj_long", 32768, HIDDEN, HIDDEN, 5, x_kind="t3",
-                   t3_channels=HIDDEN // 100)
+                   t3_channels=round(0.01 * HIDDEN))  # 72 channels
 
 # workload 6: mid-size batches between the decode and prefill regimes (the
 # 128-stream aggregate decode step and a 32-row batch), fused QKV and o_proj
