@@ -222,7 +222,7 @@ FP8BQ_API fp8bq_status fp8bq_nvfp4_gemm_a16(const void *x_bf16, const uint8_t *p
  * fp8bq_gemm without a workspace argument, for callers that cannot allocate
  * device memory: code running where no allocator is reachable (an embedding
  * runtime that hands out only fixed buffers, or a context where cudaMalloc is
- * not permitted).  The paper has no counterpart; this is a convenience of the
+ * not permitted).  The pages describe no such call; it is a convenience of the
  * library.  Same arguments, results and accuracy as fp8bq_gemm, minus the
  * workspace.  Its scratch is a 4 MiB array inside the library (held on every
  * GPU that loads it until the process exits).  Problems whose split-K scratch
