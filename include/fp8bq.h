@@ -25,8 +25,11 @@
  *
  * Ownership: the caller allocates and frees every buffer (inputs, outputs and
  * workspace) in device memory of the current device; the library never
- * allocates device memory and keeps no per-buffer state on the host (TMA
- * descriptors are encoded on every call and passed by value to the kernels).
+ * allocates device memory.  The only host state is a bounded cache of encoded
+ * TMA descriptors keyed on address, shape, element type, box and swizzle (an
+ * entry describes any tensor with that key, whatever the memory holds, so it
+ * never goes stale; fp8bq_clear_cache() empties it).  Descriptors are passed
+ * by value to the kernels.
  *
  * Execution: every compute call is asynchronous on the given stream (a
  * cudaStream_t passed as void*; NULL = the legacy default stream) and returns
@@ -41,7 +44,8 @@
  *   M, N, K <= 2^31 - 1 and every tensor smaller than 2^40 bytes (UNSUPPORTED_SHAPE);
  *   non-NULL pointers for every non-empty tensor (INVALID_ARG);
  *   every pointer 16-byte aligned (MISALIGNED);
- *   workspace at least fp8bq_workspace_size(...) bytes (WORKSPACE).
+ *   where a workspace is required (decode GEMMs and the fused linear, see
+ *     fp8bq_workspace_size), at least that many bytes (WORKSPACE).
  * Inputs must be finite; NaN or infinite inputs give unspecified codes.
  *
  * Thread safety: calls on different streams may run concurrently as long as
@@ -112,7 +116,8 @@ FP8BQ_API fp8bq_status fp8bq_quantize_weight(const void *w_bf16, int64_t N, int6
  *   y_bf16 : out, BF16 [M, N]
  *   workspace, ws_bytes : device scratch of at least
  *       fp8bq_workspace_size(FP8BQ_OP_GEMM, M, N, K) bytes (may be NULL when
- *       that is 0; for M > 128 optional, see fp8bq_workspace_size).  Its contents must be the state left by
+ *       that is 0; optional for M > 128, see fp8bq_workspace_size).  Its
+ *       contents must be the state left by
  *       fp8bq_workspace_init() or by any previous successful fp8bq_gemm or
  *       fp8bq_linear call, of any shape (every successful call restores that
  *       state); calls that share a workspace must be ordered (same stream).
