@@ -455,10 +455,13 @@ constexpr size_t kPrefillTailBytes =
 constexpr int64_t kPrefillTailMinKB = 128;  // K >= 16384
 
 // Workspace fp8bq_workspace_size reports: what the GEMM requires, or for the
-// prefill path what its split-K tail can use.
-size_t gemm_ws_bytes_full(int64_t M, int64_t N) {
+// prefill path what its split-K tail can use (only at K >= 16384; whether the
+// last wave is short enough to split also depends on the SM count, which the
+// size query does not need).
+size_t gemm_ws_bytes_full(int64_t M, int64_t N, int64_t K) {
     const size_t need = gemm_ws_bytes(M, N);
-    return M > kDecodeMaxM ? std::max(need, round256(kPrefillTailBytes)) : need;
+    const bool tail = M > kDecodeMaxM && K / 128 >= kPrefillTailMinKB;
+    return tail ? std::max(need, round256(kPrefillTailBytes)) : need;
 }
 
 size_t act_ws_bytes(int64_t M, int64_t K) { return round256(M * K) + round256(M * (K / 128) * 4); }
@@ -774,8 +777,8 @@ fp8bq_status fp8bq_nvfp4_gemm_a16(const void *x_bf16, const uint8_t *packed, con
 
 size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {
     if (check_mnk(M, N, K) != FP8BQ_OK || M == 0) return 0;
-    if (op == FP8BQ_OP_GEMM) return gemm_ws_bytes_full(M, N);
-    if (op == FP8BQ_OP_LINEAR) return act_ws_bytes(M, K) + gemm_ws_bytes_full(M, N);
+    if (op == FP8BQ_OP_GEMM) return gemm_ws_bytes_full(M, N, K);
+    if (op == FP8BQ_OP_LINEAR) return act_ws_bytes(M, K) + gemm_ws_bytes_full(M, N, K);
     return 0;
 }
 

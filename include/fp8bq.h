@@ -248,10 +248,12 @@ FP8BQ_API fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, co
 /* Bytes of workspace the operation uses for this shape (0 when none, and for
  * arguments the call would reject).  Always a multiple of 256.  For M <= 128
  * the call requires at least this much.  For M > 128 (the prefill GEMM) any
- * workspace is accepted, NULL included; with at least this much, a last wave
- * of at most 16 output tiles on the persistent grid is split K-wise over more
- * CTAs (FP32 partials summed in a fixed order, so results stay deterministic
- * and within the same tolerance), which a smaller one goes without. */
+ * workspace is accepted, NULL included, and the size is 0 unless K >= 16384.
+ * There, with at least this much, a last wave of at most 16 output tiles on
+ * the persistent grid is split K-wise over more CTAs (FP32 partials summed in
+ * a fixed order, so results stay deterministic and within the same
+ * tolerance), which a smaller workspace goes without.  The fused linear adds
+ * its activation codes and scales, which it always requires. */
 FP8BQ_API size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K);
 
 /* Put a workspace into its initial state (zero-fills ws_bytes bytes on the

@@ -121,10 +121,16 @@ def test_linear_argument_errors(L):
     assert f(GOOD, GOOD, GOOD, 300, 256, 100, GOOD, GOOD, ws, None) == SHAPE
     assert f(GOOD, GOOD, None, 300, 256, 256, GOOD, GOOD, ws, None) == INVALID
     assert f(ODD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws, None) == MISALIGNED
-    # for M > 128 only the activation codes and scales are required; the rest of
-    # the reported size is the prefill GEMM's optional split-K tail
+    # for M > 128 only the activation codes and scales are required (at this K
+    # the prefill GEMM has no split-K tail to report)
+    up = lambda b: -(-b // 256) * 256                # each part padded to 256 bytes
+    assert ws == up(300 * 256) + up(300 * 2 * 4)
+    assert f(GOOD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws - 256, None) == WORKSPACE
+    # at K >= 16384 the reported size adds the optional tail, which may be left out
+    ws_long = fp8bq.workspace_size(fp8bq.OP_LINEAR, 300, 256, 16384)
     tail = 16384 + 16 * 4 * 128 * 256 * 4
-    assert f(GOOD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws - tail - 256, None) == WORKSPACE
+    assert ws_long == up(300 * 16384) + up(300 * 128 * 4) + tail
+    assert f(GOOD, GOOD, GOOD, 300, 256, 16384, GOOD, GOOD, ws_long - tail - 256, None) == WORKSPACE
     assert f(None, None, None, 0, 256, 256, None, None, 0, None) == OK
 
 
@@ -176,9 +182,12 @@ def test_workspace_sizes(L):
     assert g(0, 256, 256) == 0 and lin(0, 256, 256) == 0
     assert g(8, 200, 256) == 0 and g(8, 256, 200) == 0           # rejected shapes
     assert fp8bq.workspace_size(7, 8, 256, 256) == 0              # unknown op
-    # prefill GEMM: optional, the split-K tail's counter header + 16 x 4 partial tiles
+    # prefill GEMM: nothing required; at K >= 16384 the optional split-K tail,
+    # its counter header + 16 x 4 partial tiles
     tail = 16384 + 16 * 4 * 128 * 256 * 4
-    assert g(8192, 9216, 7168) == tail
+    assert g(8192, 9216, 7168) == 0 and g(32768, 7168, 7168) == 0
+    assert g(4096, 7168, 21504) == g(1280, 4096, 16384) == tail
+    assert g(1280, 4096, 16256) == 0
     d = g(16, 9216, 7168)
     assert d > 0 and d % 256 == 0
     # decode split-K: counters + (N/128 + 256) slots of 16 x 128 FP32 partials
@@ -187,7 +196,7 @@ def test_workspace_sizes(L):
     assert g(17, 9216, 7168) == 16384 + (72 + 256) * 32 * 128 * 4
     assert g(64, 9216, 7168) == 16384 + (72 + 256) * 64 * 128 * 4
     assert g(65, 9216, 7168) == g(128, 9216, 7168) == 16384 + (72 + 256) * 128 * 128 * 4
-    assert g(129, 9216, 7168) == tail
+    assert g(129, 9216, 7168) == 0 and g(129, 9216, 16384) == tail
     # linear adds the activation codes and scales
     assert lin(8192, 9216, 7168) >= 8192 * 7168 + 8192 * 56 * 4
     assert lin(16, 9216, 7168) >= d + 16 * 7168 + 16 * 56 * 4
