@@ -466,6 +466,15 @@ size_t gemm_ws_bytes_full(int64_t M, int64_t N, int64_t K) {
 
 size_t act_ws_bytes(int64_t M, int64_t K) { return round256(M * K) + round256(M * (K / 128) * 4); }
 
+// The fused linear's workspace holds the GEMM's part first, never shorter than
+// the counter header, then the activation codes and scales (plain scratch).
+// So the split-K counters sit at offset 0 of every workspace, whatever the
+// operation and shape, and one workspace can serve any sequence of calls.
+size_t linear_gemm_part(int64_t M, int64_t N, int64_t K, bool with_tail) {
+    const size_t g = with_tail ? gemm_ws_bytes_full(M, N, K) : gemm_ws_bytes(M, N);
+    return std::max(g, static_cast<size_t>(decode::kCounterBytes));
+}
+
 // ---------------------------------------------------------------- launches
 
 // Up to this many groups (M <= 128 at K = 7168) the shared-memory-free
@@ -778,7 +787,7 @@ fp8bq_status fp8bq_nvfp4_gemm_a16(const void *x_bf16, const uint8_t *packed, con
 size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {
     if (check_mnk(M, N, K) != FP8BQ_OK || M == 0) return 0;
     if (op == FP8BQ_OP_GEMM) return gemm_ws_bytes_full(M, N, K);
-    if (op == FP8BQ_OP_LINEAR) return act_ws_bytes(M, K) + gemm_ws_bytes_full(M, N, K);
+    if (op == FP8BQ_OP_LINEAR) return act_ws_bytes(M, K) + linear_gemm_part(M, N, K, true);
     return 0;
 }
 
@@ -812,21 +821,25 @@ fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const float *sw
     if (!x_bf16 || !qw || !sw || !y_bf16) return FP8BQ_ERR_INVALID_ARG;
     if (!aligned16(x_bf16) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16))
         return FP8BQ_ERR_MISALIGNED;
-    const size_t need = act_ws_bytes(M, K) + gemm_ws_bytes(M, N);
-    if (!workspace || ws_bytes < need) return FP8BQ_ERR_WORKSPACE;
+    const size_t act = act_ws_bytes(M, K);
+    const size_t part_req = linear_gemm_part(M, N, K, false);
+    if (!workspace || ws_bytes < act + part_req) return FP8BQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return FP8BQ_ERR_MISALIGNED;
     const DeviceInfo *d = device_info();
     if (!d) return FP8BQ_ERR_NO_DEVICE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // [GEMM part][activation codes][activation scales]; the GEMM part takes
+    // the prefill split-K tail's size when the workspace holds it
+    const size_t part_full = linear_gemm_part(M, N, K, true);
+    const size_t part = ws_bytes >= act + part_full ? part_full : part_req;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    uint8_t *qa = ws;
-    float *sa = reinterpret_cast<float *>(ws + round256(M * K));
-    void *gemm_ws = ws + act_ws_bytes(M, K);
+    uint8_t *qa = ws + part;
+    float *sa = reinterpret_cast<float *>(qa + round256(M * K));
     cudaError_t e = launch_quantize_act(*d, x_bf16, M, K, qa, sa, s);
     if (e != cudaSuccess) return FP8BQ_ERR_CUDA;
     fp8bq_status err;
-    e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, gemm_ws, ws_bytes - act_ws_bytes(M, K), s,
-                    &err, /*early_weights=*/true);
+    e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, ws, part, s, &err,
+                    /*early_weights=*/true);
     if (err != FP8BQ_OK) return err;
     return from_cuda(e);
 }

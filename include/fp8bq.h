@@ -252,8 +252,13 @@ FP8BQ_API fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, co
  * There, with at least this much, a last wave of at most 16 output tiles on
  * the persistent grid is split K-wise over more CTAs (FP32 partials summed in
  * a fixed order, so results stay deterministic and within the same
- * tolerance), which a smaller workspace goes without.  The fused linear adds
- * its activation codes and scales, which it always requires. */
+ * tolerance), which a smaller workspace goes without.  The fused linear
+ * requires, besides the GEMM's part (never less than its 16 KB counter
+ * header), its activation codes and scales.
+ * Every workspace starts with the same 16 KB header of split-K counters, at
+ * offset 0 for both operations and every shape, and every successful call
+ * leaves them at zero: one workspace, large enough for each call, can serve
+ * any sequence of fp8bq_gemm and fp8bq_linear calls in stream order. */
 FP8BQ_API size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K);
 
 /* Put a workspace into its initial state (zero-fills ws_bytes bytes on the

@@ -121,16 +121,18 @@ def test_linear_argument_errors(L):
     assert f(GOOD, GOOD, GOOD, 300, 256, 100, GOOD, GOOD, ws, None) == SHAPE
     assert f(GOOD, GOOD, None, 300, 256, 256, GOOD, GOOD, ws, None) == INVALID
     assert f(ODD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws, None) == MISALIGNED
-    # for M > 128 only the activation codes and scales are required (at this K
+    # for M > 128: the 16 KB counter header (kept at offset 0 of every
+    # workspace), then the activation codes and scales, all required (at this K
     # the prefill GEMM has no split-K tail to report)
     up = lambda b: -(-b // 256) * 256                # each part padded to 256 bytes
-    assert ws == up(300 * 256) + up(300 * 2 * 4)
+    assert ws == 16384 + up(300 * 256) + up(300 * 2 * 4)
     assert f(GOOD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws - 256, None) == WORKSPACE
-    # at K >= 16384 the reported size adds the optional tail, which may be left out
+    # at K >= 16384 the optional tail (header included) replaces the bare header
     ws_long = fp8bq.workspace_size(fp8bq.OP_LINEAR, 300, 256, 16384)
     tail = 16384 + 16 * 4 * 128 * 256 * 4
-    assert ws_long == up(300 * 16384) + up(300 * 128 * 4) + tail
-    assert f(GOOD, GOOD, GOOD, 300, 256, 16384, GOOD, GOOD, ws_long - tail - 256, None) == WORKSPACE
+    assert ws_long == tail + up(300 * 16384) + up(300 * 128 * 4)
+    assert f(GOOD, GOOD, GOOD, 300, 256, 16384, GOOD, GOOD, ws_long - tail + 16384 - 256,
+             None) == WORKSPACE
     assert f(None, None, None, 0, 256, 256, None, None, 0, None) == OK
 
 
@@ -179,6 +181,7 @@ def test_nvfp4_argument_errors(L):
 def test_workspace_sizes(L):
     g = lambda M, N, K: fp8bq.workspace_size(fp8bq.OP_GEMM, M, N, K)
     lin = lambda M, N, K: fp8bq.workspace_size(fp8bq.OP_LINEAR, M, N, K)
+    up = lambda b: -(-b // 256) * 256
     assert g(0, 256, 256) == 0 and lin(0, 256, 256) == 0
     assert g(8, 200, 256) == 0 and g(8, 256, 200) == 0           # rejected shapes
     assert fp8bq.workspace_size(7, 8, 256, 256) == 0              # unknown op
@@ -197,9 +200,11 @@ def test_workspace_sizes(L):
     assert g(64, 9216, 7168) == 16384 + (72 + 256) * 64 * 128 * 4
     assert g(65, 9216, 7168) == g(128, 9216, 7168) == 16384 + (72 + 256) * 128 * 128 * 4
     assert g(129, 9216, 7168) == 0 and g(129, 9216, 16384) == tail
-    # linear adds the activation codes and scales
-    assert lin(8192, 9216, 7168) >= 8192 * 7168 + 8192 * 56 * 4
-    assert lin(16, 9216, 7168) >= d + 16 * 7168 + 16 * 56 * 4
+    # linear adds the activation codes and scales to the GEMM's part, which is
+    # never less than the counter header
+    assert lin(8192, 9216, 7168) == 16384 + 8192 * 7168 + 8192 * 56 * 4
+    assert lin(16, 9216, 7168) == d + 16 * 7168 + up(16 * 56 * 4)
+    assert lin(4096, 7168, 21504) == tail + 4096 * 21504 + 4096 * 168 * 4
     for args in ((1, 128, 128), (17, 384, 1024), (4096, 7168, 21504)):
         assert lin(*args) % 256 == 0 and g(*args) % 256 == 0
 

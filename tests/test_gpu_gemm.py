@@ -385,6 +385,38 @@ def test_gemm_workspace_reused_across_calls():
     assert torch.equal(outs[0].view(torch.int16), outs[3].view(torch.int16))
 
 
+def test_one_workspace_serves_gemm_and_linear_of_any_shape():
+    # The split-K counters sit at offset 0 of every workspace, and the fused
+    # linear keeps its activation scratch behind them: one workspace serves a
+    # mixed sequence of linear and gemm calls (stream-K decode, cluster decode,
+    # mid-size M, the prefill split-K tail) in stream order.
+    calls = [("linear", 4, 19200, 512), ("gemm", 3, 32768, 256), ("linear", 8, 9216, 7168),
+             ("gemm", 4, 19200, 512), ("linear", 100, 1152, 7168), ("linear", 1280, 4096, 16384),
+             ("gemm", 3, 32768, 256), ("gemm", 1280, 4096, 16384), ("linear", 4, 19200, 512)]
+    op_of = {"linear": fp8bq.OP_LINEAR, "gemm": fp8bq.OP_GEMM}
+    size = max(fp8bq.workspace_size(op_of[op], M, N, K) for op, M, N, K in calls)
+    ws = torch.zeros(size, dtype=torch.uint8, device="cuda")
+    first = {}
+    for op, M, N, K in calls:
+        x, qa, sa, qw, sw = operands(M, N, K, 500 + M + K)
+        if op == "linear":
+            y = fp8bq.linear(x.cuda(), to_dev_codes(qw), to_dev_f32(sw), workspace=ws)
+        else:
+            y = fp8bq.gemm(to_dev_codes(qa), to_dev_f32(sa), to_dev_codes(qw), to_dev_f32(sw),
+                           workspace=ws)
+        torch.cuda.synchronize()
+        rows = sample_rows(M, 24, extra=(1024, 1151)) if M > 128 else np.arange(M, dtype=np.int64)
+        ref = (oracle.linear_ref(x, qw, sw, rows=rows) if op == "linear"
+               else oracle.gemm_ref(qa, sa, qw, sw, rows=rows))
+        check(bf16_to_f64(y)[rows], ref)
+        key = (op, M, N, K)
+        if key in first:
+            assert torch.equal(first[key].view(torch.int16), y.cpu().view(torch.int16))
+        first.setdefault(key, y.cpu())
+    assert fp8bq.last_device_status() == 0
+    assert int(ws[:16384].sum()) == 0  # every counter back at zero
+
+
 @pytest.mark.parametrize("M", [4, 333])
 def test_device_chain_without_host_sync(M):
     # weight and activation quantization feed the GEMM on one stream with no host
