@@ -235,3 +235,35 @@ def test_binding_fails_loudly_without_cuda_tensors():
     x = torch.zeros(4, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fp8bq.quantize_act(x)
+
+
+def test_header_compiles_as_c_and_cxx_and_links(L, tmp_path):
+    # A C11 client: the header alone, strict warnings, every declared function
+    # referenced and linked against the library, and calls that need no device.
+    refs = "\n".join(f"    (void)&{n};" for n in declared_functions())
+    src = tmp_path / "client.c"
+    src.write_text(f"""#include "fp8bq.h"
+#include <stdio.h>
+#include <string.h>
+int main(void) {{
+{refs}
+    if (fp8bq_version() <= 0) return 1;
+    if (strcmp(fp8bq_status_string(FP8BQ_OK), "ok") != 0) return 2;
+    if (fp8bq_workspace_size(FP8BQ_OP_GEMM, 16, 9216, 7168) == 0) return 3;
+    if (fp8bq_gemm(NULL, NULL, NULL, NULL, 8, 200, 256, NULL, NULL, 0, NULL)
+        != FP8BQ_ERR_UNSUPPORTED_SHAPE) return 4;
+    if (fp8bq_quantize_act(NULL, 4, 128, NULL, NULL, NULL) != FP8BQ_ERR_INVALID_ARG) return 5;
+    puts("client ok");
+    return 0;
+}}
+""")
+    libdir = os.path.dirname(fp8bq.LIB_PATH)
+    exe = tmp_path / "client"
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.dirname(HEADER), str(src), "-o", str(exe), f"-L{libdir}",
+                    "-lfp8bq", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and "client ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
+    # the same header in a C++ translation unit (extern "C" linkage)
+    subprocess.run(["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-fsyntax-only",
+                    "-x", "c++", HEADER], check=True)
