@@ -82,8 +82,8 @@ def test_gemm_decode_path(M, N, K):
 # several n-blocks split across CTAs and a K long enough that the staged scales
 # cut the ring to four stages at M > 64
 MIDM_SHAPES = [(17, 128, 128), (32, 256, 384), (33, 1024, 7168), (64, 384, 1024),
-               (65, 2048, 896), (100, 1152, 7168), (128, 256, 256), (128, 512, 21504),
-               (40, 20480, 256), (128, 19200, 384)]
+               (65, 2048, 896), (100, 1152, 7168), (127, 384, 1024), (128, 256, 256),
+               (128, 512, 21504), (40, 20480, 256), (128, 19200, 384)]
 
 
 @pytest.mark.parametrize("M,N,K", MIDM_SHAPES)
@@ -96,7 +96,7 @@ def test_gemm_mid_m_decode_path(M, N, K):
 # M > 128 (the 129..256 rows of the mid-size range included) runs on the prefill kernel
 PREFILL_SHAPES = [(129, 384, 1024), (200, 2048, 7168), (255, 1152, 512), (256, 1024, 1024),
                   (255, 9216, 256), (300, 1152, 512),
-                  (1000, 512, 896), (300, 128, 7168), (2048, 2048, 384)]
+                  (1000, 512, 896), (300, 128, 7168), (2048, 2048, 384), (8191, 384, 256)]
 
 
 @pytest.mark.parametrize("M,N,K", PREFILL_SHAPES)
