@@ -194,6 +194,13 @@ def test_linear_matches_oracle_and_unfused_path(M, N, K):
     gq, gs = fp8bq.quantize_act(xd)
     y2 = fp8bq.gemm(gq, gs, to_dev_codes(qw), to_dev_f32(sw))
     assert torch.equal(y.t.view(torch.int16), y2.view(torch.int16))
+    # the linear's scratch (behind the GEMM's part of a workspace of the
+    # reported size) holds exactly those codes and scales
+    up = lambda b: -(-b // 256) * 256
+    off = ws.numel() - up(M * K) - up(M * (K // 128) * 4)
+    assert torch.equal(ws[off:off + M * K].view(M, K), gq)
+    so = off + up(M * K)
+    assert torch.equal(ws[so:so + M * (K // 128) * 4].view(torch.float32).view(M, K // 128), gs)
 
 
 # ------------------------------------------------------------------ prefill split-K tail
