@@ -17,7 +17,9 @@ Each check is chosen so that a plausible slip in the oracle fails it:
   shapes, including the 128x128x128 brute force, with the FP64 summation
   error bound; identity and permuted one-hot weights in closed form; an
   exact-arithmetic regime where FP64 must be exact; M = 1 as numpy's dot.
-* BF16 rounding: torch's RNE cast on binary32-representable values.
+* BF16 rounding: torch's RNE cast on binary32-representable values, and exact
+  rational rounding on FP64 values just off the BF16 midpoints (which a
+  version that rounds through binary32 first gets wrong).
 """
 import math
 
@@ -347,3 +349,73 @@ def test_bf16_round_matches_torch_on_float32_values():
     ref = bits(torch.from_numpy(v).to(torch.bfloat16))
     got = oracle.bf16_round(v.astype(np.float64))
     assert np.array_equal(got, ref)
+
+
+def _bf16_bits_exact(v: float) -> int:
+    """BF16 bit pattern of a double by exact rational arithmetic: the significand
+    rounded to 8 bits, ties to even, with the BF16 subnormal quantum 2^-133 below
+    2^-126 and infinity from 2^128 on (the definition of round-to-nearest-even on
+    the bfloat16 grid: 1 sign, 8 exponent, 7 fraction bits)."""
+    from fractions import Fraction
+    sign = 0x8000 if math.copysign(1.0, v) < 0 else 0
+    a = Fraction(abs(v))
+    if a == 0:
+        return sign
+    e = math.floor(math.log2(abs(v)))
+    if Fraction(2) ** e > a:           # log2 rounded up at an exact power boundary
+        e -= 1
+    if Fraction(2) ** (e + 1) <= a:
+        e += 1
+    e = max(e, -126)
+    quantum = Fraction(2) ** (e - 7)
+    q = a / quantum
+    fl = q.numerator // q.denominator
+    rem = q - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    r = fl * quantum
+    if r >= Fraction(2) ** 128:
+        return sign | 0x7F80
+    if r < Fraction(2) ** -126:        # subnormal: fraction field counts 2^-133 steps
+        return sign | int(r / Fraction(2) ** -133)
+    ex = math.floor(math.log2(float(r)))
+    frac = int((r / Fraction(2) ** ex - 1) * 128)
+    return sign | ((ex + 127) << 7) | frac
+
+
+def test_bf16_round_on_float64_values_off_the_midpoints():
+    """Values that are not binary32: BF16 midpoints moved by 2^-30 .. 2^-40 relative
+    (above and below), both signs, across normal binades, the subnormal range and
+    the overflow edge, against exact rational rounding.  Rounding through binary32
+    first (double rounding) lands most of these on the midpoint itself and then
+    ties to even, so it must disagree on them: checked below with torch's cast."""
+    rng = np.random.default_rng(7)
+    vals = []
+    for _ in range(600):
+        e = int(rng.integers(-125, 127))
+        frac = int(rng.integers(0, 128))
+        mid = (1.0 + (frac + 0.5) / 128.0) * 2.0 ** e      # a BF16 midpoint (exact in FP64)
+        d = 2.0 ** -int(rng.integers(30, 41))
+        vals += [mid * (1 + d), mid * (1 - d)]
+    for k in range(0, 128, 5):                             # subnormal midpoints (k + 1/2) 2^-133
+        mid = (k + 0.5) * 2.0 ** -133
+        vals += [mid * (1 + 2.0 ** -35), mid * (1 - 2.0 ** -35)]
+    top = (2.0 - 2.0 ** -8) * 2.0 ** 127                   # midpoint between BF16 max and 2^128
+    vals += [top * (1 - 2.0 ** -33), top * (1 + 2.0 ** -33), top, (2.0 - 2.0 ** -7) * 2.0 ** 127]
+    vals += [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 2.0 ** -126 * (1 - 2.0 ** -40)]
+    v = np.array(vals + [-x for x in vals], dtype=np.float64)
+    assert not np.array_equal(v.astype(np.float32).astype(np.float64), v)   # truly FP64 inputs
+    ref = np.array([_bf16_bits_exact(float(x)) for x in v], dtype=np.uint16)
+    assert np.array_equal(oracle.bf16_round(v), ref)
+    # the inputs tell a double-rounding implementation apart from the right one
+    twice = bits(torch.from_numpy(v).to(torch.float32).to(torch.bfloat16))
+    assert (twice != ref).sum() > len(v) // 4
+
+
+def test_bf16_exact_reference_agrees_with_torch_on_float32_values():
+    """The rational reference above, checked where torch's cast is single rounding."""
+    rng = np.random.default_rng(3)
+    v = np.concatenate([rng.standard_normal(300).astype(np.float32) * 1e3,
+                        np.float32([1e-40, -2.5e-39, 3e38, 1.0 + 2 ** -8])])
+    ref = bits(torch.from_numpy(v).to(torch.bfloat16))
+    assert np.array_equal(np.array([_bf16_bits_exact(float(x)) for x in v], np.uint16), ref)
