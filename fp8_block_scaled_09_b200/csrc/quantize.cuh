@@ -27,19 +27,52 @@ __device__ __forceinline__ float scale_from_amax_bits(uint32_t amax_bits) {
     return amax_bits == 0 ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax_bits), 448.0f);
 }
 
+// Smallest scale for which the corrected quotient below reproduces the E4M3
+// code of fl32(x / scale) for every BF16 x with |x| <= 448 scale (checked for
+// every BF16 amax down to this bound and every such x; below about 2^-110 the
+// residual r is no longer exact).  Smaller scales use the IEEE division.
+constexpr float kCorrectedQuotientMinScale = 0x1p-92f;
+
+// x / s from y = RN(1/s) by one FMA correction step (Markstein's theorem,
+// IBM J. Res. Dev. 34(1), 1990; Muller et al., "Handbook of Floating-Point
+// Arithmetic", on division with a fused multiply-add): with q = RN(x y), the
+// residual r = x - q s is exact, and RN(q + r y) is the correctly rounded
+// quotient while no intermediate underflows.  The sign of x is put back so an
+// exact zero keeps it (-0 / s must give the code 0x80).
+__device__ __forceinline__ float corrected_quotient(float x, float s, float y) {
+    const float q = __fmul_rn(x, y);
+    const float r = __fmaf_rn(-q, s, x);
+    return copysignf(__fmaf_rn(r, y, q), x);
+}
+
 // Eight BF16 values (one 16-byte vector) -> eight E4M3 codes (8 bytes): each
 // code is the saturating round-to-nearest conversion of the IEEE quotient
-// fl32(x / scale).  (Division-free schemes that reproduce these codes exactly
-// -- a reciprocal with a rounding-interval check -- were measured and were
-// slower here than __fdiv_rn.)
-__device__ __forceinline__ uint2 encode8(uint4 v, float scale) {
+// fl32(x / scale).  The quotient comes from one reciprocal per call and three
+// FP operations per element (corrected_quotient), which gives fl32(x / scale)
+// bit for bit wherever |x / scale| >= 2^-11 or x = +-0, and the same code
+// everywhere else; tiny scales take the IEEE division.
+// encode8 with the reciprocal y = RN(1 / scale) supplied by the caller (used
+// only when scale >= kCorrectedQuotientMinScale), for callers that encode many
+// vectors with one scale.
+__device__ __forceinline__ uint2 encode8_y(uint4 v, float scale, float y) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t c[4];
+    if (scale >= kCorrectedQuotientMinScale) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        c[i] = e4m3x2_satfinite(__fdiv_rn(__uint_as_float(w[i] << 16), scale),
-                                __fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), scale));
+        for (int i = 0; i < 4; ++i)
+            c[i] = e4m3x2_satfinite(corrected_quotient(__uint_as_float(w[i] << 16), scale, y),
+                                    corrected_quotient(__uint_as_float(w[i] & 0xFFFF0000u), scale, y));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            c[i] = e4m3x2_satfinite(__fdiv_rn(__uint_as_float(w[i] << 16), scale),
+                                    __fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), scale));
+    }
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+__device__ __forceinline__ uint2 encode8(uint4 v, float scale) {
+    return encode8_y(v, scale, __frcp_rn(scale));
 }
 
 __device__ __forceinline__ uint32_t amax_bits8(uint4 v) {
