@@ -6,8 +6,10 @@ GEMV set: fp8bq_linear (dynamic group-128 activation quantization fused into
 the call, block-scaled FP8 GEMM, BF16 out) for M in {1, 4, 8} tokens against
 the fused QKV weight [9216, 7168] and the o_proj weight [7168, 7168] -- six
 linear layers per step.  The weights are quantized once (the offline half of
-the method) and rotated over four device copies per shape so that every step
-streams them from HBM (4 x 66 MB and 4 x 51 MB, larger than the 126 MB L2).
+the method) and every call of a step reads its own device copy: six copies per
+shape, steps alternating between copies 0-2 and 3-5, so a copy is read again
+only after two whole steps (more than 350 MB of other weights, well over the
+126 MB L2) and every call streams its weights from HBM.
 
 ``value`` is algorithmic HBM bytes per second (weight codes + weight scales +
 BF16 activations + BF16 outputs; one pass over each), timed with CUDA events
@@ -23,7 +25,9 @@ around CUDA-graph replays of the steps, max over ranks.  Alongside:
 * ``workloads``  GEMM-kernel and linear throughput for every other shape.
 * ``e2e``        the same decode steps through the public API from pinned host
                  buffers: H2D copy of X, the linear call, D2H copy of Y.
-* ``cpu_baseline`` the CPU oracle (plain C, FP64 GEMM) on full decode steps.
+* ``cpu_baseline`` the CPU oracle (plain C, FP64 GEMM) on full decode steps;
+                 each prefill row also carries one, timed on two row subsets
+                 and extrapolated to the full M (labelled as such).
 
 ``--impl reference`` times the CPU oracle instead, on the same metric.
 ``--gpus N`` (under torchrun) runs N independent replicas, one per GPU: the
@@ -49,12 +53,17 @@ import workloads as W  # noqa: E402
 
 METRIC = "FP8 block-scaled GEMM TFLOPS (prefill) & HBM GB/s (decode), % of roofline, 1 B200"
 FP8_OVER_BF16 = 2.0          # nominal dense ratio 4.5 / 2.25 PFLOP/s
-ROTATE = 4                   # device copies of each decode weight
-# DRAM bytes (read + write) of one decode GEMM launch, o_proj M=1 (7168 x 7168), from the ncu
-# capture summarised in profiles/gemm_decode_kernel_o_proj_m1.md; scaled to other shapes by
-# their algorithmic bytes (the capture shows DRAM bytes = algorithmic bytes within 0.04%).
-DECODE_TRAFFIC_CAPTURE = {"shape": (1, 7168, 7168), "dram_bytes": 51_472_896 + 5_888,
-                          "source": "profiles/gemm_decode_kernel_o_proj_m1.md"}
+COPIES = 6                   # device copies of each decode weight (3 calls per shape per step)
+STEP_VARIANTS = 2            # steps alternate between copies 0-2 and 3-5
+# DRAM bytes (read + write) per decode GEMM launch, averaged over consecutive launches of the
+# graph-replayed decode-GEMM step (per-call weight copies, L2 state carried from launch to
+# launch), measured by ncu on `bench.py --only decode-graph`.  Valid only for the decode
+# kernel source it was taken on: `kernel_sha` is the SHA-256 (first 16 hex digits) of
+# gemm_decode.cuh + ptx.cuh; when the source differs, the traffic is reported as null.
+DECODE_TRAFFIC = {"bytes_per_launch": None, "kernel_sha": None,
+                  "how": "ncu --cache-control none --clock-control none --metrics "
+                         "dram__bytes_read.sum,dram__bytes_write.sum on the graph-replayed "
+                         "decode GEMM launches of one bench step (6 launches)"}
 DECODE_WORKLOAD = ("decode GEMV set: fp8bq_linear, M in {1,4,8} x {fused QKV W[9216,7168], "
                    "o_proj W[7168,7168]}, E4M3 128x128-blocked weights, X BF16 N(0,1) with "
                    "7 outlier channels x20")
@@ -71,6 +80,21 @@ def load_peaks() -> dict:
                 "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
+
+
+def decode_kernel_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm_decode.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "fp8_block_scaled_09_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def weight_copy(step: int, call: int) -> int:
+    """Device copy of its shape's weight that `call` (0..2 within its shape) of
+    step `step` reads: steps alternate between copies 0-2 and 3-5."""
+    return 3 * (step % STEP_VARIANTS) + call
 
 
 def linear_bytes(g: W.Gemm) -> int:
@@ -280,6 +304,50 @@ def run_reference(args, rank: int, world: int) -> None:
 
 # ----------------------------------------------------------------------------- our arm
 
+def decode_device_set(torch, fp8bq, dev, xs_host, ws_host):
+    """Device weights (COPIES per shape), activations, codes and workspaces of the
+    decode set; each call records its index among the calls of its shape."""
+    qw_rot, sw_rot = {}, {}
+    for N, w in ws_host.items():
+        qw, sw = fp8bq.quantize_weight(w.to(dev))
+        qw_rot[N] = [qw] + [qw.clone() for _ in range(COPIES - 1)]
+        sw_rot[N] = [sw] + [sw.clone() for _ in range(COPIES - 1)]
+    calls, seen = [], {}
+    for g, xh in zip(W.DECODE_SET, xs_host):
+        x = xh.to(dev)
+        qa, sa = fp8bq.quantize_act(x)
+        calls.append({
+            "g": g, "x": x, "qa": qa, "sa": sa, "call": seen.get(g.N, 0),
+            "y": torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev),
+            "ws_lin": fp8bq.new_workspace(fp8bq.OP_LINEAR, g.M, g.N, g.K, dev),
+            "ws_gemm": fp8bq.new_workspace(fp8bq.OP_GEMM, g.M, g.N, g.K, dev),
+            "x_host": xh,
+        })
+        seen[g.N] = seen.get(g.N, 0) + 1
+    assert all(v * STEP_VARIANTS <= COPIES for v in seen.values())
+    return qw_rot, sw_rot, calls
+
+
+def decode_gemm_step(fp8bq, calls, qw_rot, sw_rot, r: int) -> None:
+    """The decode GEMM kernel alone on every call of step r (pre-quantized activations)."""
+    for c in calls:
+        k = weight_copy(r, c["call"])
+        N = c["g"].N
+        fp8bq.gemm(c["qa"], c["sa"], qw_rot[N][k], sw_rot[N][k], out=c["y"],
+                   workspace=c["ws_gemm"])
+
+
+def capture_steps(torch, step_fn):
+    """One CUDA graph per step variant (steps alternate between weight copies)."""
+    graphs = []
+    for r in range(STEP_VARIANTS):
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph):
+            step_fn(r)
+        graphs.append(gph)
+    return graphs
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     import torch
     import torch.distributed as dist
@@ -301,35 +369,18 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
 
     # ---------------------------------------------------------------- decode set
     xs_host, ws_host = decode_host_inputs()
-    qw_rot, sw_rot = {}, {}
-    for N, w in ws_host.items():
-        qw, sw = fp8bq.quantize_weight(w.to(dev))
-        qw_rot[N] = [qw] + [qw.clone() for _ in range(ROTATE - 1)]
-        sw_rot[N] = [sw] + [sw.clone() for _ in range(ROTATE - 1)]
-    calls = []
-    for g, xh in zip(W.DECODE_SET, xs_host):
-        x = xh.to(dev)
-        qa, sa = fp8bq.quantize_act(x)
-        calls.append({
-            "g": g, "x": x, "qa": qa, "sa": sa,
-            "y": torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev),
-            "ws_lin": fp8bq.new_workspace(fp8bq.OP_LINEAR, g.M, g.N, g.K, dev),
-            "ws_gemm": fp8bq.new_workspace(fp8bq.OP_GEMM, g.M, g.N, g.K, dev),
-            "x_host": xh,
-        })
+    qw_rot, sw_rot, calls = decode_device_set(torch, fp8bq, dev, xs_host, ws_host)
     step_bytes = sum(linear_bytes(c["g"]) for c in calls)
     gemm_step_bytes = sum(gemm_bytes(c["g"]) for c in calls)
 
     def linear_step(r: int):
         for c in calls:
+            k = weight_copy(r, c["call"])
             N = c["g"].N
-            fp8bq.linear(c["x"], qw_rot[N][r], sw_rot[N][r], out=c["y"], workspace=c["ws_lin"])
+            fp8bq.linear(c["x"], qw_rot[N][k], sw_rot[N][k], out=c["y"], workspace=c["ws_lin"])
 
     def gemm_step(r: int):
-        for c in calls:
-            N = c["g"].N
-            fp8bq.gemm(c["qa"], c["sa"], qw_rot[N][r], sw_rot[N][r], out=c["y"],
-                       workspace=c["ws_gemm"])
+        decode_gemm_step(fp8bq, calls, qw_rot, sw_rot, r)
 
     # eager warm-up (also sets the library up on this device), launch counts per step
     n0 = fp8bq.launch_count()
@@ -340,45 +391,35 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     gemm_kernels_per_step = fp8bq.launch_count() - n0
     torch.cuda.synchronize()
 
-    def capture(step_fn):
-        graphs = []
-        for r in range(ROTATE):
-            gph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gph):
-                step_fn(r)
-            graphs.append(gph)
-        return graphs
-
-    lin_graphs = capture(linear_step)
-    gemm_graphs = capture(gemm_step)
+    lin_graphs = capture_steps(torch, linear_step)
+    gemm_graphs = capture_steps(torch, gemm_step)
     for i in range(warmup):
-        lin_graphs[i % ROTATE].replay()
+        lin_graphs[i % STEP_VARIANTS].replay()
     torch.cuda.synchronize()
 
     barrier()
     with clocks:
-        ms = events_ms(torch, lambda i: lin_graphs[i % ROTATE].replay(), args.steps)
+        ms = events_ms(torch, lambda i: lin_graphs[i % STEP_VARIANTS].replay(), args.steps)
     barrier()
     ms = max_over_ranks(ms, world, dev)
     value = replica_throughput(world, step_bytes, args.steps, ms)
 
     # dominant kernel: the decode GEMM alone
     for i in range(warmup):
-        gemm_graphs[i % ROTATE].replay()
+        gemm_graphs[i % STEP_VARIANTS].replay()
     barrier()
     with clocks:
-        gms = events_ms(torch, lambda i: gemm_graphs[i % ROTATE].replay(), args.steps)
+        gms = events_ms(torch, lambda i: gemm_graphs[i % STEP_VARIANTS].replay(), args.steps)
     barrier()
     gms = max_over_ranks(gms, world, dev)
     gemm_launches = args.steps * gemm_kernels_per_step
     gemm_gbs = gemm_step_bytes * args.steps / (gms * 1e-3) / 1e9
-    cap_M, cap_N, cap_K = DECODE_TRAFFIC_CAPTURE["shape"]
-    cap_ratio = DECODE_TRAFFIC_CAPTURE["dram_bytes"] / gemm_bytes(W.Gemm("capture", cap_M, cap_N, cap_K, 0))
-    traffic = cap_ratio * gemm_step_bytes / gemm_kernels_per_step
+    sha = decode_kernel_sha()
+    traffic = DECODE_TRAFFIC["bytes_per_launch"] if DECODE_TRAFFIC["kernel_sha"] == sha else None
     roofline = {"bound": "hbm", "achieved": gemm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": traffic,
-                "traffic_source": f"ncu dram read+write of one launch ({DECODE_TRAFFIC_CAPTURE['source']}),"
-                                  " scaled to this mix by algorithmic bytes",
+                "traffic_source": DECODE_TRAFFIC["how"] if traffic is not None else
+                                  f"null: no capture for this decode kernel source ({sha})",
                 "kernel": "fp8bq::decode::gemm_decode_kernel<16> (cluster split)",
                 "avg_launch_us": gms * 1e3 / gemm_launches,
                 "algorithmic_bytes_per_launch": gemm_step_bytes / gemm_kernels_per_step,
@@ -406,16 +447,17 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     def e2e_step(r: int):
         x_all.copy_(x_all_pin, non_blocking=True)
         for c in calls:
+            k = weight_copy(r, c["call"])
             N = c["g"].N
-            fp8bq.linear(c["x_e2e"], qw_rot[N][r], sw_rot[N][r], out=c["y_e2e"],
+            fp8bq.linear(c["x_e2e"], qw_rot[N][k], sw_rot[N][k], out=c["y_e2e"],
                          workspace=c["ws_lin"])
         y_all_pin.copy_(y_all, non_blocking=True)
 
     for i in range(warmup):
-        e2e_step(i % ROTATE)
+        e2e_step(i)
     barrier()
     with clocks:
-        ems = events_ms(torch, lambda i: e2e_step(i % ROTATE), args.steps)
+        ems = events_ms(torch, lambda i: e2e_step(i), args.steps)
     barrier()
     ems = max_over_ranks(ems, world, dev)
     h2d = x_all.numel() * 2
@@ -429,7 +471,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     extras = {}
     if not args.quick:
         extras = prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_sus,
-                                       args)
+                                       args, cpu=rank == 0 and world == 1 and not args.no_cpu_baseline)
 
     status = fp8bq.last_device_status()
     if status != 0:
@@ -448,8 +490,9 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
             "config": {"workload": DECODE_WORKLOAD, "layers_per_step": len(calls),
                        "algorithmic_bytes_per_step": step_bytes,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": f"inputs larger than L2: weights rotated over {ROTATE} device "
-                             "copies per shape",
+                       "l2": f"inputs larger than L2: each call of a step reads its own weight "
+                             f"copy ({COPIES} per shape); a copy is read again only after two "
+                             "whole steps (> 350 MB of other weights)",
                        "timing": "CUDA events around CUDA-graph replays, max over ranks"},
             "roofline": roofline,
             "cpu_baseline": cpu,
@@ -462,14 +505,41 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         print(json.dumps(line), flush=True)
 
 
-def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_sus, args):
+def oracle_prefill_baseline(g: W.Gemm, x_host, w_host) -> dict:
+    """The CPU oracle's linear layer (quantize the activation rows, FP64 GEMM) on
+    two evenly spaced row subsets of a prefill shape, all N and K, extrapolated to
+    the full M with t(M) = a + b M fitted to the two timings (a: the per-call
+    dequantization of W; b: one row).  The weight quantization is offline and
+    untimed, as on the GPU."""
+    import oracle
+    oracle.build()
+    qw, sw = oracle.quantize_weight(w_host)
+    times = {}
+    for r in (8, 24):
+        rows = np.linspace(0, g.M - 1, r).round().astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.linear_ref(x_host, qw, sw, rows=rows)
+        times[r] = time.perf_counter() - t0
+    b = max(1e-12, (times[24] - times[8]) / 16)
+    a = max(0.0, times[8] - 8 * b)
+    t_full = a + b * g.M
+    return {"value": g.flops / t_full / 1e12, "unit": "TFLOP/s",
+            "cores": len(os.sched_getaffinity(0)), "kind": "oracle", "extrapolated": True,
+            "sample": f"oracle.linear_ref on 8 and 24 evenly spaced rows of {g.M} (all N, K): "
+                      f"{times[8]:.2f} s and {times[24]:.2f} s; full M extrapolated as "
+                      f"a + b M = {t_full:.1f} s"}
+
+
+def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_sus, args,
+                          cpu: bool = False):
     iters = max(5, min(20, args.steps))
     warm = 3
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     out = {}
 
     def shape_result(g: W.Gemm, with_linear: bool):
-        x = g.make_x().to(dev)
+        x_host = g.make_x()
+        x = x_host.to(dev)
         qw, sw = fp8bq.quantize_weight(g.make_w().to(dev))
         qa, sa = fp8bq.quantize_act(x)
         y = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
@@ -497,6 +567,8 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
             if tl:
                 ml = statistics.fmean(tl)
                 r.update({"linear_us": ml * 1e3, "linear_tflops": g.flops / (ml * 1e-3) / 1e12})
+            if cpu:
+                r["cpu_baseline"] = oracle_prefill_baseline(g, x_host, g.make_w())
         del x, qw, sw, qa, sa, y
         return r
 
@@ -505,7 +577,7 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
         "workload": "prefill fused QKV: X[8192,7168] x W[9216,7168]^T, BF16 out",
         "metric": "TFLOP/s (2 M N K)", "linear_tflops": pq["linear_tflops"],
         "linear_us": pq["linear_us"], "gemm_tflops": pq["gemm_tflops"],
-        "gemm_us": pq["gemm_us"],
+        "gemm_us": pq["gemm_us"], "cpu_baseline": pq.get("cpu_baseline"),
         "roofline": {"bound": "tensor", "achieved": pq["gemm_tflops"], "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": pq["gemm_tflops"] / fp8_peak,
                      "frac_of_sustained": pq["gemm_tflops"] / fp8_peak_sus, "traffic": None,
@@ -585,6 +657,38 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
         "unfused_us": mu * 1e3,
         "unfused": "torch silu * up into BF16 h, then fp8bq.quantize_act(h): context only"}
     del gu, qh, sh, hb
+
+    # gate/up GEMM -> codes of the down projection's input: the fused epilogue
+    # (fp8bq_gemm_silu_mul_quantize) against the GEMM writing BF16 gate/up and
+    # the SiLU kernel reading it back (drafter MLP shape, M = 4096, I = 8192)
+    g = W.DRAFTER_GATE_UP
+    I = g.N // 2
+    xg = g.make_x().to(dev)
+    qwg, swg = fp8bq.quantize_weight(g.make_w().to(dev))
+    qag, sag = fp8bq.quantize_act(xg)
+    gu = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
+    qh = torch.empty((g.M, I), dtype=torch.uint8, device=dev)
+    sh = torch.empty((g.M, I // 128), dtype=torch.float32, device=dev)
+    wsg = fp8bq.new_workspace(fp8bq.OP_GEMM, g.M, g.N, g.K, dev)
+
+    def chain():
+        fp8bq.gemm(qag, sag, qwg, swg, out=gu, workspace=wsg)
+        fp8bq.silu_mul_quantize(gu, qh, sh)
+
+    with clocks:
+        tfu = flushed_ms(torch, lambda: fp8bq.gemm_silu_mul_quantize(qag, sag, qwg, swg, q=qh, s=sh),
+                         iters, warm, flush)
+        tch = flushed_ms(torch, chain, iters, warm, flush)
+    mfu, mch = statistics.fmean(tfu), statistics.fmean(tch)
+    out["gate_up_silu"] = {
+        "workload": "drafter gate/up X[4096,7168] x W[16384,7168]^T -> E4M3 codes and scales of "
+                    "h = silu(gate) * up [4096, 8192] (the down projection's input)",
+        "fused_us": mfu * 1e3, "fused_tflops": g.flops / (mfu * 1e-3) / 1e12,
+        "fused_frac_fp8": g.flops / (mfu * 1e-3) / 1e12 / fp8_peak,
+        "chain_us": mch * 1e3,
+        "chain": "fp8bq_gemm (BF16 gate/up to HBM) then fp8bq_silu_mul_quantize",
+        "timing": f"mean of {iters} graph replays, CUDA events, L2 flushed before each"}
+    del xg, qwg, swg, qag, sag, gu, qh, sh, wsg
 
     # NVFP4 weight-only GEMM (A16), decode shapes: back-to-back graph replays over 4
     # weight copies per shape (larger than L2), like the headline decode measurement
@@ -678,6 +782,15 @@ def run_profile_case(case: str) -> None:
         gu = torch.randn((4096, 16384), device=dev).mul_(2).to(torch.bfloat16)
         for _ in range(3):
             fp8bq.silu_mul_quantize(gu)
+    elif case == "decode-graph":
+        # the bench's decode-GEMM step: per-call weight copies, CUDA-graph replays
+        xs_host, ws_host = decode_host_inputs()
+        qw_rot, sw_rot, calls = decode_device_set(torch, fp8bq, dev, xs_host, ws_host)
+        decode_gemm_step(fp8bq, calls, qw_rot, sw_rot, 0)
+        torch.cuda.synchronize()
+        graphs = capture_steps(torch, lambda r: decode_gemm_step(fp8bq, calls, qw_rot, sw_rot, r))
+        for i in range(4):
+            graphs[i % STEP_VARIANTS].replay()
     else:
         gs = {"decode": W.DECODE_SET, "midm": W.MIDM_SET}.get(case, (W.PREFILL_QKV,))
         wq = {}
@@ -707,8 +820,8 @@ def main() -> None:
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--quick", action="store_true", help="decode set only (no prefill/workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=("decode", "midm", "prefill", "quantize", "kv", "silu",
-                                       "nvfp4"),
+    ap.add_argument("--only", choices=("decode", "decode-graph", "midm", "prefill", "quantize",
+                                       "kv", "silu", "nvfp4"),
                     help="profiling case: run one kernel family a few times, print a short line")
     args = ap.parse_args()
 

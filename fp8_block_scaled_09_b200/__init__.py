@@ -29,13 +29,15 @@ import torch
 __all__ = [
     "Fp8bqError", "lib", "quantize_act", "quantize_weight", "gemm", "gemm_noalloc", "linear",
     "workspace_size", "new_workspace", "workspace_init", "last_device_status",
-    "launch_count", "status_string", "selftest_timeout", "OP_GEMM", "OP_LINEAR", "LIB_PATH",
-    "kv_write_e4m3", "silu_mul_quantize", "nvfp4_quantize_weight", "nvfp4_gemm_a16",
+    "launch_count", "status_string", "selftest_timeout", "OP_GEMM", "OP_LINEAR", "OP_GEMM_SILU",
+    "LIB_PATH", "kv_write_e4m3", "silu_mul_quantize", "gemm_silu_mul_quantize",
+    "nvfp4_quantize_weight", "nvfp4_gemm_a16",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bq.so")
 OP_GEMM = 0
 OP_LINEAR = 1
+OP_GEMM_SILU = 2
 
 STATUS_NAMES = {
     0: "FP8BQ_OK", 1: "FP8BQ_ERR_INVALID_ARG", 2: "FP8BQ_ERR_UNSUPPORTED_SHAPE",
@@ -75,6 +77,7 @@ def lib() -> ctypes.CDLL:
         L.fp8bq_selftest_timeout.argtypes = [ctypes.c_uint32, P]
         L.fp8bq_kv_write_e4m3.argtypes = [P, P, I, I, I, P, P, P, I, I, P]
         L.fp8bq_silu_mul_quantize.argtypes = [P, I, I, P, P, P, P]
+        L.fp8bq_gemm_silu_mul_quantize.argtypes = [P, P, P, P, I, I, I, P, P, P, P, S, P]
         L.fp8bq_nvfp4_quantize_weight.argtypes = [P, I, I, P, P, P, P]
         L.fp8bq_nvfp4_gemm_a16.argtypes = [P, P, P, P, I, I, I, P, P]
         L.fp8bq_workspace_size.argtypes = [ctypes.c_int, I, I, I]
@@ -92,6 +95,7 @@ def lib() -> ctypes.CDLL:
         for name in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
                      "fp8bq_workspace_init", "fp8bq_last_device_status", "fp8bq_gemm_noalloc",
                      "fp8bq_selftest_timeout", "fp8bq_kv_write_e4m3", "fp8bq_silu_mul_quantize",
+                     "fp8bq_gemm_silu_mul_quantize",
                      "fp8bq_nvfp4_quantize_weight", "fp8bq_nvfp4_gemm_a16"):
             getattr(L, name).restype = st
         _lib = L
@@ -299,6 +303,42 @@ def silu_mul_quantize(gu: torch.Tensor, q: torch.Tensor | None = None, s: torch.
         _need(h, torch.bfloat16, "h")
     _check(lib().fp8bq_silu_mul_quantize(_ptr(gu), M, I, _ptr(q), _ptr(s), _ptr(h), _stream(gu)),
            "fp8bq_silu_mul_quantize")
+    return q, s
+
+
+def gemm_silu_mul_quantize(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+                           q: torch.Tensor | None = None, s: torch.Tensor | None = None,
+                           h: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """fp8bq_gemm_silu_mul_quantize: the gate/up GEMM (fused weight codes qw [2I, K],
+    gate rows first) with the SiLU-gated product quantized in its epilogue ->
+    (codes uint8 [M, I], scales FP32 [M, I/128]), the same as
+    silu_mul_quantize(gemm(qa, sa, qw, sw)).  Pass h (BF16 [M, I]) to also receive h."""
+    qa, qw = _codes(qa), _codes(qw)
+    _need(qa, torch.uint8, "qa")
+    _need(qw, torch.uint8, "qw")
+    _need(sa, torch.float32, "sa")
+    _need(sw, torch.float32, "sw")
+    M, K = qa.shape
+    two_i = qw.shape[0]
+    if two_i % 2:
+        raise ValueError("qw must have an even number of rows (gate | up)")
+    I = two_i // 2
+    if q is None:
+        q = torch.empty((M, I), dtype=torch.uint8, device=qa.device)
+    if s is None:
+        s = torch.empty((M, I // 128 if I % 128 == 0 else 0), dtype=torch.float32, device=qa.device)
+    q = _codes(q)
+    _need(q, torch.uint8, "q")
+    _need(s, torch.float32, "s")
+    if h is not None:
+        _need(h, torch.bfloat16, "h")
+    if workspace is None:
+        workspace = new_workspace(OP_GEMM_SILU, M, two_i, K, qa.device)
+    _check(lib().fp8bq_gemm_silu_mul_quantize(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), M, I, K,
+                                              _ptr(q), _ptr(s), _ptr(h), _ptr(workspace),
+                                              workspace.numel(), _stream(qa)),
+           "fp8bq_gemm_silu_mul_quantize")
     return q, s
 
 

@@ -19,9 +19,15 @@
 //                       registers, CUDA-core FMA); larger M: nvfp4::nvfp4_gemm_a16_kernel
 //                       (BF16 dequant into shared memory + tcgen05 kind::f16)
 //   silu_mul_quantize-> silu_mul_quantize_kernel (half-warp per 128-channel group)
-//   linear           -> quantize_act into the workspace, then the gemm path; the
-//                       decode kernel then streams its first weight blocks while
-//                       the quantizer still runs (programmatic dependent launch)
+//   gemm_silu_mul_quantize -> M > 128: prefill::gemm_prefill_kernel<256, true>
+//                       (gate/up GEMM whose epilogue quantizes silu(gate) * up);
+//                       smaller M: the decode GEMM, then silu_mul_quantize
+//   linear, M <= 128 -> quantize_act into the workspace, then the decode GEMM,
+//                       which streams its first weight blocks while the
+//                       quantizer still runs (programmatic dependent launch)
+//   linear, M > 128  -> one launch: prefill::gemm_prefill_kernel<256, false, true>
+//                       quantizes X into the workspace while its GEMM consumes
+//                       the finished chunks
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -114,6 +120,18 @@ EncodeTiledFn encode_fn() {
     return g_encode;
 }
 
+// Sets the prefill kernel variant's shared-memory limit and checks that it was
+// built with the register count its setmaxnreg split assumes.
+template <bool kSilu, bool kFusedAct>
+bool prefill_variant_ready() {
+    auto *k = prefill::gemm_prefill_kernel<kPrefillBN, kSilu, kFusedAct>;
+    cudaFuncAttributes fa;
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                prefill::Layout<kPrefillBN, kSilu, kFusedAct>::kDynamicSmem) ==
+               cudaSuccess &&
+           cudaFuncGetAttributes(&fa, k) == cudaSuccess && fa.numRegs == prefill::kLaunchRegs;
+}
+
 // Current device's info, set up once per device (kernel attributes, status word).
 const DeviceInfo *device_info() {
     int dev = -1;
@@ -129,16 +147,12 @@ const DeviceInfo *device_info() {
         if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), g_status) != cudaSuccess)
             return;
         if (cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess) return;
-        if (cudaFuncSetAttribute(prefill::gemm_prefill_kernel<kPrefillBN>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 prefill::Layout<kPrefillBN>::kDynamicSmem) != cudaSuccess)
-            return;
         // The prefill kernel moves registers between warpgroups with setmaxnreg;
         // the split is only safe if the launch allocates exactly what it was
         // designed for (otherwise setmaxnreg.inc could wait forever).
         cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, prefill::gemm_prefill_kernel<kPrefillBN>) != cudaSuccess ||
-            fa.numRegs != prefill::kLaunchRegs)
+        if (!prefill_variant_ready<false, false>() || !prefill_variant_ready<true, false>() ||
+            !prefill_variant_ready<false, true>())
             return;
         // CTA-pair prefill kernel: optional; any failure here only leaves it off.
         d.pair_clusters = 0;
@@ -454,6 +468,21 @@ constexpr size_t kPrefillTailBytes =
 
 constexpr int64_t kPrefillTailMinKB = 128;  // K >= 16384
 
+// Split-K tail parts of the prefill kernel for a grid over `tiles` tiles (0:
+// no split): a last wave of at most kTailMaxTiles tiles leaves most SMs idle,
+// so each of its tiles is split K-wise into up to kTailMaxParts parts.
+// Measured: it pays for long K (M=4096, N=7168: K=21504 681 -> 631 us) but not
+// for K=8192 (269 -> 278 us), where the partial hand-off outweighs it.
+int prefill_tail_parts(int64_t tiles, int grid, int64_t KB, const void *ws, size_t ws_bytes) {
+    const int64_t rest = tiles % grid;
+    int parts = 0;
+    if (ws != nullptr && aligned16(ws) && ws_bytes >= kPrefillTailBytes && tiles > grid && rest >= 1 &&
+        rest <= prefill::kTailMaxTiles && KB >= kPrefillTailMinKB)
+        parts = static_cast<int>(std::min<int64_t>(std::min<int64_t>(prefill::kTailMaxParts, grid / rest), KB));
+    return parts < 2 ? 0 : parts;
+}
+
+
 // Workspace fp8bq_workspace_size reports: what the GEMM requires, or for the
 // prefill path what its split-K tail can use (only at K >= 16384; whether the
 // last wave is short enough to split also depends on the SM count, which the
@@ -464,7 +493,15 @@ size_t gemm_ws_bytes_full(int64_t M, int64_t N, int64_t K) {
     return tail ? std::max(need, round256(kPrefillTailBytes)) : need;
 }
 
-size_t act_ws_bytes(int64_t M, int64_t K) { return round256(M * K) + round256(M * (K / 128) * 4); }
+// The linear's activation scratch: codes [M, K], then scales.  For M > 128 the
+// scales are stored transposed, [K/128, m_pad] with M rounded up to 128 rows
+// (the single-launch prefill linear reads one 512-byte strip per K chunk).
+int64_t act_scale_rows(int64_t M) {
+    return M > kDecodeMaxM ? (M + prefill::BM - 1) / prefill::BM * prefill::BM : M;
+}
+size_t act_ws_bytes(int64_t M, int64_t K) {
+    return round256(M * K) + round256(act_scale_rows(M) * (K / 128) * 4);
+}
 
 // The fused linear's workspace holds the GEMM's part first, never shorter than
 // the counter header, then the activation codes and scales (plain scratch).
@@ -568,27 +605,88 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
         }
         const int64_t tiles = ((M + prefill::BM - 1) / prefill::BM) * ((N + kPrefillBN - 1) / kPrefillBN);
         const int grid = static_cast<int>(tiles < d.sm_count ? tiles : d.sm_count);
-        // A last wave of at most kTailMaxTiles tiles leaves most SMs idle: split
-        // each of its tiles K-wise into up to kTailMaxParts parts.  Measured: it
-        // pays for long K (M=4096, N=7168: K=21504 681 -> 631 us) but not for
-        // K=8192 (269 -> 278 us), where the partial hand-off outweighs it.
-        const int64_t KB = K / 128, rest = tiles % grid;
-        int tail_parts = 0;
-        if (ws != nullptr && aligned16(ws) && ws_bytes >= kPrefillTailBytes && tiles > grid && rest >= 1 &&
-            rest <= prefill::kTailMaxTiles && KB >= kPrefillTailMinKB)
-            tail_parts = static_cast<int>(std::min<int64_t>(
-                std::min<int64_t>(prefill::kTailMaxParts, grid / rest), KB));
-        if (tail_parts < 2) tail_parts = 0;
+        const int tail_parts = prefill_tail_parts(tiles, grid, K / 128, ws, ws_bytes);
         int *tail_counters = tail_parts ? static_cast<int *>(ws) : nullptr;
         float *tail_partials =
             tail_parts ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes)
                        : nullptr;
-        return launch(prefill::gemm_prefill_kernel<kPrefillBN>, dim3(grid),
-                      dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN>::kDynamicSmem, st,
-                      ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
-                      static_cast<int>(N), static_cast<int>(K), d.status, tail_parts, tail_partials,
-                      tail_counters);
+        return launch(prefill::gemm_prefill_kernel<kPrefillBN, false, false>, dim3(grid),
+                      dim3(prefill::kNumThreads),
+                      prefill::Layout<kPrefillBN, false, false>::kDynamicSmem, st, ta, tb, sa, sw,
+                      static_cast<__nv_bfloat16 *>(y), static_cast<int>(M), static_cast<int>(N),
+                      static_cast<int>(K), d.status, tail_parts, tail_partials, tail_counters,
+                      prefill::SiluOut{nullptr, nullptr, nullptr}, ta, prefill::FusedAct{});
     }
+}
+
+// Whether the single-launch linear (activation quantization inside the
+// prefill GEMM) takes this shape: its completion counters must fit in the
+// workspace's counter header.
+bool fused_prefill_linear_fits(int64_t M, int64_t K) {
+    const int64_t groups = ((M + prefill::BM - 1) / prefill::BM + prefill::kGroupM - 1) / prefill::kGroupM;
+    return M > kDecodeMaxM && prefill::kActCtrBase + groups * (K / 128) <= prefill::kActClaimSlot;
+}
+
+// The linear layer for M > 128 in one launch: the prefill kernel quantizes X
+// into the workspace (codes qa [M, K], scales transposed saT [K/128, m_pad])
+// while it runs the GEMM on what is done.  ws: the workspace (its counter
+// header at offset 0); part: bytes of its GEMM part.
+cudaError_t launch_linear_prefill(const DeviceInfo &d, const void *x, const uint8_t *qw,
+                                  const float *sw, int64_t M, int64_t N, int64_t K, void *y,
+                                  void *ws, size_t part, uint8_t *qa, float *saT, cudaStream_t st,
+                                  fp8bq_status *err) {
+    *err = FP8BQ_OK;
+    CUtensorMap ta, tb, tx;
+    if (!make_tmap(&ta, qa, M, K, prefill::BM) || !make_tmap(&tb, qw, N, K, kPrefillBN) ||
+        !make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, prefill::BK / 2,
+                      prefill::BM, CU_TENSOR_MAP_SWIZZLE_128B)) {
+        *err = FP8BQ_ERR_CUDA;
+        return cudaSuccess;
+    }
+    const int64_t tiles = ((M + prefill::BM - 1) / prefill::BM) * ((N + kPrefillBN - 1) / kPrefillBN);
+    const int grid = static_cast<int>(tiles < d.sm_count ? tiles : d.sm_count);
+    const int tail_parts = prefill_tail_parts(tiles, grid, K / 128, ws, part);
+    int *ctr = static_cast<int *>(ws);
+    float *tail_partials =
+        tail_parts ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes) : nullptr;
+    const int m_pad = static_cast<int>((M + prefill::BM - 1) / prefill::BM * prefill::BM);
+    return launch(prefill::gemm_prefill_kernel<kPrefillBN, false, true>, dim3(grid),
+                  dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN, false, true>::kDynamicSmem,
+                  st, ta, tb, static_cast<const float *>(saT), sw, static_cast<__nv_bfloat16 *>(y),
+                  static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), d.status, tail_parts,
+                  tail_partials, tail_parts ? ctr : static_cast<int *>(nullptr),
+                  prefill::SiluOut{nullptr, nullptr, nullptr}, tx,
+                  prefill::FusedAct{qa, saT, ctr, m_pad});
+}
+
+// Gate/up GEMM with the SiLU-gated product quantized in its epilogue (M > 128):
+// the prefill kernel with tiles of 128 gate and the same 128 up channels.
+cudaError_t launch_gemm_silu(const DeviceInfo &d, const uint8_t *qa, const float *sa,
+                             const uint8_t *qw, const float *sw, int64_t M, int64_t I, int64_t K,
+                             uint8_t *q, float *s, void *h, cudaStream_t st, fp8bq_status *err) {
+    *err = FP8BQ_OK;
+    CUtensorMap ta, tb;
+    if (!make_tmap(&ta, qa, M, K, prefill::BM) || !make_tmap(&tb, qw, 2 * I, K, 128)) {
+        *err = FP8BQ_ERR_CUDA;
+        return cudaSuccess;
+    }
+    const int64_t tiles = ((M + prefill::BM - 1) / prefill::BM) * (I / 128);
+    const int grid = static_cast<int>(tiles < d.sm_count ? tiles : d.sm_count);
+    return launch(prefill::gemm_prefill_kernel<kPrefillBN, true, false>, dim3(grid),
+                  dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN, true, false>::kDynamicSmem,
+                  st, ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(nullptr), static_cast<int>(M),
+                  static_cast<int>(2 * I), static_cast<int>(K), d.status, 0,
+                  static_cast<float *>(nullptr), static_cast<int *>(nullptr),
+                  prefill::SiluOut{q, s, static_cast<__nv_bfloat16 *>(h)}, ta, prefill::FusedAct{});
+}
+
+// Workspace of the gate/up GEMM with the SiLU epilogue: none on the fused
+// path (M > 128); otherwise the decode GEMM's, then the BF16 gate/up output
+// [M, 2I] that the separate SiLU kernel reads.
+size_t silu_ws_bytes(int64_t M, int64_t I) {
+    if (M > kDecodeMaxM) return 0;
+    return std::max(gemm_ws_bytes(M, 2 * I), static_cast<size_t>(decode::kCounterBytes)) +
+           round256(M * 2 * I * 2);
 }
 
 }  // namespace
@@ -602,9 +700,28 @@ namespace fp8bq {
 namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-void *g_noalloc_ptr[kMaxDevices];
-cudaError_t g_noalloc_err[kMaxDevices];
-std::once_flag g_noalloc_once[kMaxDevices];
+// Device address of the array per device, kept once a lookup has succeeded; a
+// failed lookup is not remembered, so a later call tries again.
+std::atomic<void *> g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// The array's device address on device `dev` (current), or null.  In host code
+// the array's name is only a host-side stand-in, never a device address.
+void *noalloc_scratch(int dev) {
+    void *p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (p != nullptr) return p;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    p = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess && p != nullptr) {
+            g_noalloc_ptr[dev].store(p, std::memory_order_release);
+        } else {
+            p = nullptr;
+            cudaGetLastError();  // leave no error behind for the caller's next CUDA call
+        }
+    }
+    return p;
+}
 }  // namespace
 }  // namespace fp8bq
 
@@ -788,6 +905,7 @@ size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {
     if (check_mnk(M, N, K) != FP8BQ_OK || M == 0) return 0;
     if (op == FP8BQ_OP_GEMM) return gemm_ws_bytes_full(M, N, K);
     if (op == FP8BQ_OP_LINEAR) return act_ws_bytes(M, K) + linear_gemm_part(M, N, K, true);
+    if (op == FP8BQ_OP_GEMM_SILU) return N % 256 == 0 ? silu_ws_bytes(M, N / 2) : 0;
     return 0;
 }
 
@@ -835,13 +953,53 @@ fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const float *sw
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint8_t *qa = ws + part;
     float *sa = reinterpret_cast<float *>(qa + round256(M * K));
+    fp8bq_status err;
+    if (fused_prefill_linear_fits(M, K)) {
+        cudaError_t e = launch_linear_prefill(*d, x_bf16, qw, sw, M, N, K, y_bf16, ws, part, qa, sa, s,
+                                              &err);
+        if (err != FP8BQ_OK) return err;
+        return from_cuda(e);
+    }
     cudaError_t e = launch_quantize_act(*d, x_bf16, M, K, qa, sa, s);
     if (e != cudaSuccess) return FP8BQ_ERR_CUDA;
-    fp8bq_status err;
     e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, ws, part, s, &err,
                     /*early_weights=*/true);
     if (err != FP8BQ_OK) return err;
     return from_cuda(e);
+}
+
+fp8bq_status fp8bq_gemm_silu_mul_quantize(const uint8_t *qa, const float *sa, const uint8_t *qw,
+                                           const float *sw, int64_t M, int64_t I, int64_t K,
+                                           uint8_t *q_e4m3, float *s, void *h_bf16, void *workspace,
+                                           size_t ws_bytes, void *stream) {
+    if (I <= 0 || I % 128 != 0 || I > kMaxDim / 2) return FP8BQ_ERR_UNSUPPORTED_SHAPE;
+    fp8bq_status st = check_mnk(M, 2 * I, K);
+    if (st != FP8BQ_OK) return st;
+    if (M == 0) return FP8BQ_OK;
+    if (!qa || !sa || !qw || !sw || !q_e4m3 || !s) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) ||
+        !aligned16(q_e4m3) || !aligned16(s) || (h_bf16 != nullptr && !aligned16(h_bf16)))
+        return FP8BQ_ERR_MISALIGNED;
+    const size_t need = silu_ws_bytes(M, I);
+    if (need && (!workspace || ws_bytes < need)) return FP8BQ_ERR_WORKSPACE;
+    if (need && !aligned16(workspace)) return FP8BQ_ERR_MISALIGNED;
+    const DeviceInfo *d = device_info();
+    if (!d) return FP8BQ_ERR_NO_DEVICE;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    fp8bq_status err;
+    if (M > kDecodeMaxM) {
+        cudaError_t e = launch_gemm_silu(*d, qa, sa, qw, sw, M, I, K, q_e4m3, s, h_bf16, cs, &err);
+        if (err != FP8BQ_OK) return err;
+        return from_cuda(e);
+    }
+    // Decode-sized M: the decode GEMM writes the BF16 gate/up output into the
+    // workspace behind its own part, then the SiLU kernel quantizes it.
+    const size_t part = need - round256(M * 2 * I * 2);
+    void *gu = static_cast<uint8_t *>(workspace) + part;
+    cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, 2 * I, K, gu, workspace, part, cs, &err);
+    if (err != FP8BQ_OK) return err;
+    if (e != cudaSuccess) return FP8BQ_ERR_CUDA;
+    return fp8bq_silu_mul_quantize(gu, M, I, q_e4m3, s, h_bf16, stream);
 }
 
 fp8bq_status fp8bq_workspace_init(void *workspace, size_t ws_bytes, void *stream) {
@@ -914,21 +1072,19 @@ fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, const uint8_
     const DeviceInfo *d = device_info();
     if (!d) return FP8BQ_ERR_NO_DEVICE;
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FP8BQ_ERR_CUDA;
-    // Once per device, with that device current: the array's device address.
-    // (In host code the array's name is only a host-side stand-in.)
-    std::call_once(g_noalloc_once[dev], [dev] {
-        g_noalloc_err[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
-    });
-    if (g_noalloc_err[dev] != cudaSuccess || g_noalloc_ptr[dev] == nullptr) return FP8BQ_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8BQ_ERR_CUDA;
+    // With the device current: the array's device address (looked up on the
+    // first call that succeeds in doing so on this device).
+    void *scratch = noalloc_scratch(dev);
+    if (scratch == nullptr) return FP8BQ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // The array keeps whatever the previous call left; the split-K counters
     // must start at zero, so clear them on this call's stream first.
-    if (need && cudaMemsetAsync(g_noalloc_ptr[dev], 0, static_cast<size_t>(decode::kCounterBytes),
-                                s) != cudaSuccess)
+    if (need && cudaMemsetAsync(scratch, 0, static_cast<size_t>(decode::kCounterBytes), s) !=
+                    cudaSuccess)
         return FP8BQ_ERR_CUDA;
     fp8bq_status err;
-    cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, g_noalloc_ptr[dev],
+    cudaError_t e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, scratch,
                                 /*ws_bytes (no prefill tail split)=*/0, s, &err,
                                 /*early_weights=*/false, /*allow_decode=*/fits);
     if (err != FP8BQ_OK) return err;

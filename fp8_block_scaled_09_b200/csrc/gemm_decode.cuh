@@ -54,6 +54,8 @@ namespace fp8bq {
 namespace decode {
 
 constexpr int BNW = 128;  // weight rows per unit (one scale block)
+// Suspend hint of this kernel's barrier waits (see mbar_wait).
+constexpr uint32_t kDecodeSuspendNs = 10000;
 constexpr int BK = 128;
 constexpr int kMaxMT = 128;
 constexpr int kMaxGrid = 256;  // workspace is sized for at most this many CTAs
@@ -112,11 +114,18 @@ struct Layout {
     }
 };
 
+// Rows of the staged activation-scale table: one per K block the CTA's unit
+// range touches, i.e. min(KB, units); the range's K blocks form one cyclic
+// interval starting at u_begin mod KB.
+__host__ __device__ inline int64_t scale_rows(int64_t KB, int64_t units_per_cta_max) {
+    return units_per_cta_max < KB ? units_per_cta_max : KB;
+}
+
 // Dynamic shared memory for a launch (1 KB of it for the alignment of the ring).
 template <int MT>
 __host__ __device__ inline int64_t smem_bytes(int stages, int64_t KB, int64_t units_per_cta_max) {
-    return Layout<MT>::scale_off(stages) + Layout<MT>::kSaRow * KB * 4 + (units_per_cta_max + 1) * 4 +
-           1024;
+    return Layout<MT>::scale_off(stages) + Layout<MT>::kSaRow * scale_rows(KB, units_per_cta_max) * 4 +
+           (units_per_cta_max + 1) * 4 + 1024;
 }
 
 // Bytes of one ring slot for a token tile.
@@ -213,7 +222,10 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     }
     const int64_t n_steps = (u_end - u_begin + kStep - 1) / kStep;
     constexpr int kSaRow = Layout::kSaRow;
-    float *sw_s = sa_s + kSaRow * KB;  // sw[u] for u in [u_begin, u_end): sw is [NB, KB] row-major
+    // staged activation scales: row r holds K block (kb_first + r) mod KB
+    const int kb_first = static_cast<int>(u_begin % KB);
+    const int sa_rows = static_cast<int>(scale_rows(KB, u_end - u_begin));
+    float *sw_s = sa_s + kSaRow * sa_rows;  // sw[u] for u in [u_begin, u_end): sw is [NB, KB] row-major
 
     allow_dependent_launch();
     if (threadIdx.x == 0) {
@@ -284,7 +296,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
             uint32_t phase = n_early == kStages ? 1u : 0u;
             int64_t issued = n_early;
             for (int64_t i = n_early; i < n_steps; ++i) {
-                if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) break;
+                if (!mbar_wait<false, kDecodeSuspendNs>(&empty[stage], phase ^ 1, abort_flag, status)) break;
                 const int cnt = step_units(i);
                 uint8_t *st = smem + stage * Layout::kStage;
                 mbar_arrive_expect_tx(&full[stage], cnt * Layout::kUnit);
@@ -302,7 +314,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 }
             }
             for (int64_t i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-                mbar_wait(&full[i % kStages], static_cast<uint32_t>((i / kStages) & 1), nullptr,
+                mbar_wait<false, kDecodeSuspendNs>(&full[i % kStages], static_cast<uint32_t>((i / kStages) & 1), nullptr,
                           status);
         }
     } else if (warp == 1) {
@@ -310,8 +322,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
             const uint32_t idesc = umma_idesc_e4m3(BNW, MT);
             uint32_t stage = 0, phase = 0, grp = 0, gphase = 0;
             for (int64_t i = 0; i < n_steps; ++i) {
-                if (!mbar_wait(&tempty[grp], gphase ^ 1, abort_flag, status) ||
-                    !mbar_wait(&full[stage], phase, abort_flag, status))
+                if (!mbar_wait<false, kDecodeSuspendNs>(&tempty[grp], gphase ^ 1, abort_flag, status) ||
+                    !mbar_wait<false, kDecodeSuspendNs>(&full[stage], phase, abort_flag, status))
                     break;
                 tc_fence_after_sync();
                 const int cnt = step_units(i);
@@ -336,7 +348,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 }
             }
             umma_commit(drain);
-            mbar_wait(drain, 0, nullptr, status);
+            mbar_wait<false, kDecodeSuspendNs>(drain, 0, nullptr, status);
         }
     } else if (warp < kSplitWarp) {
         const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
@@ -349,12 +361,13 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         // async copies keep all of them in flight at once.  A warp copies a
         // tile of 8 k-blocks x 4 tokens: four 32-byte global segments, and 32
         // distinct shared-memory banks since kSaRow is 4 times an odd number.
-        const int kb_tiles = (KB + 7) / 8;
+        const int kb_tiles = (sa_rows + 7) / 8;
         for (int t = ptid >> 5; t < kb_tiles * (MT / 4); t += kPromoWarps) {
-            const int kb = (t % kb_tiles) * 8 + (lane & 7);
+            const int r = (t % kb_tiles) * 8 + (lane & 7);
             const int m = (t / kb_tiles) * 4 + (lane >> 3);
-            if (kb < KB) {
-                float *dst = sa_s + kb * kSaRow + m;
+            if (r < sa_rows) {
+                const int kb = kb_first + r < KB ? kb_first + r : kb_first + r - KB;
+                float *dst = sa_s + r * kSaRow + m;
                 if (m < M)
                     cp_async_4(dst, sa + static_cast<int64_t>(m) * KB + kb);
                 else
@@ -378,7 +391,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
             const int j = static_cast<int>((u - u_begin) % kStep);  // unit within its step
             const bool last_of_step = j == kStep - 1 || u == u_end - 1;
             if (j == 0) {
-                if (!mbar_wait(&tfull[grp], gphase, abort_flag, status)) break;
+                if (!mbar_wait<false, kDecodeSuspendNs>(&tfull[grp], gphase, abort_flag, status)) break;
                 tc_fence_after_sync();
             }
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
@@ -400,7 +413,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                     gphase ^= 1;
                 }
             }
-            const float4 *sa4 = reinterpret_cast<const float4 *>(sa_s + kb * kSaRow + col0);
+            const int sa_r = kb >= kb_first ? kb - kb_first : kb - kb_first + KB;
+            const float4 *sa4 = reinterpret_cast<const float4 *>(sa_s + sa_r * kSaRow + col0);
 #pragma unroll
             for (int i = 0; i < kCols / 4; ++i) {
                 const float4 a = sa4[i];
@@ -450,7 +464,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         for (int i = 0; i < 2; ++i) {
             if (i >= plan.count) break;
             const int nb = plan.nb[i];
-            if (!mbar_wait(&flushed[i], 0, abort_flag, status)) break;
+            if (!mbar_wait<false, kDecodeSuspendNs>(&flushed[i], 0, abort_flag, status)) break;
             if (lane == 0) {
                 const int c_first = cta_of_unit(static_cast<int64_t>(nb) * KB, U, G);
                 const int c_last = cta_of_unit(static_cast<int64_t>(nb) * KB + KB - 1, U, G);

@@ -34,6 +34,8 @@
 #include <stdint.h>
 
 #include "ptx.cuh"
+#include "quantize.cuh"
+#include "silu_quant.cuh"
 
 namespace fp8bq {
 namespace prefill {
@@ -49,24 +51,111 @@ constexpr int kProducerRegs = 40;    // warpgroup 0 after setmaxnreg.dec
 constexpr int kConsumerRegs = 232;   // warpgroups 1-2 after setmaxnreg.inc
 static_assert(128 * kProducerRegs + 256 * kConsumerRegs <= kNumThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
+// With the activation quantizer in warpgroup 0 (kFusedAct), that warpgroup
+// keeps more registers: at 40 its encode loop spilled and ran ~10x slower.
+constexpr int kProducerRegsFused = 72;
+constexpr int kConsumerRegsFused = 216;
+static_assert(128 * kProducerRegsFused + 256 * kConsumerRegsFused <= kNumThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr int kFirstPromoWarp = 4;
 constexpr int kPromoWarps = 8;
 constexpr int kGroupM = 16;
 constexpr int kScaleLookahead = 2;   // K chunks of scale prefetch in registers
 
-template <int BN>
+// Activation quantization inside the GEMM launch (kFusedAct, the linear
+// layer): scale strips of kSaRing chunks in flight, and a two-slot ring of
+// 128 x 128 BF16 activation chunks for the quantizer warp.
+constexpr int kSaRing = 8;
+constexpr int kSaStrip = BM * 4;           // 128 activation scales of one chunk
+constexpr int kQChunkBytes = BM * BK * 2;  // 32 KB of BF16
+constexpr int kQSlots = 2;
+
+template <int BN, bool kSilu = false, bool kFusedAct = false>
 struct Layout {
     static_assert(BN == 256, "tile width");
     static constexpr int kA = BM * BK;
     static constexpr int kB = BN * BK;
     static constexpr int kStage = kA + kB;
     static constexpr int kBarOff = kStages * kStage;
-    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tfull, tempty, drain
+    // full, empty (per stage), tfull, tempty, drain; kFusedAct: sfull, sempty
+    // (per scale strip), qfull (per quantizer slot)
+    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + (kFusedAct ? 2 * kSaRing + kQSlots : 0);
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kBytes = kMiscOff + 16;
+    // SiLU epilogue: per-row group maxima of the two column halves, two tiles
+    // deep, each a 64-bit word tagged with the tile's index
+    static constexpr int kXchgOff = kMiscOff + 32;
+    static constexpr int kXchgBytes = kSilu ? 2 * BM * 2 * 8 : 0;
+    static constexpr int kSaOff = (kXchgOff + kXchgBytes + 1023) & ~1023;
+    static constexpr int kQOff = kSaOff + (kFusedAct ? kSaRing * kSaStrip : 0);
+    static constexpr int kBytes = kQOff + (kFusedAct ? kQSlots * kQChunkBytes : 0);
     static constexpr int kDynamicSmem = kBytes + 1024;  // room to align the base to 1024 B
+    static_assert(kDynamicSmem <= 227 * 1024, "shared memory");
     static constexpr uint32_t kTmemCols = 2 * BN;
 };
+
+// Header slots (int32, in the counter header at the start of the workspace)
+// used by the in-launch activation quantization: one completion counter per
+// (group of kGroupM m-tiles, K chunk) from kActCtrBase on, the chunk claim
+// counter and the CTA exit counter in the last two slots.  The last CTA to
+// exit zeroes them all again.
+constexpr int kActCtrBase = 64;
+constexpr int kHeaderInts = 4096;
+constexpr int kActClaimSlot = kHeaderInts - 2;
+constexpr int kActExitSlot = kHeaderInts - 1;
+
+struct FusedAct {
+    uint8_t *qa;   // codes [M, K] (workspace)
+    float *saT;    // scales transposed [K/128, m_pad] (workspace)
+    int *ctr;      // the workspace's counter header
+    int m_pad;     // M rounded up to a multiple of 128
+};
+
+// Relaxed (no ordering) load of a global int.
+__device__ __forceinline__ int ld_relaxed_gpu(const int *p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Orders this thread's generic-proxy global accesses with its later
+// async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Producer side of the in-launch quantization: returns once the activation
+// chunks [0, kb] of an m-tile group are all quantized (counter == gm), reading
+// up to eight counters at once and remembering in `ready_upto` the longest
+// prefix seen complete.  Bounded like every wait.  Acquires on success.
+__device__ __forceinline__ bool wait_act_chunks(const int *ctr, int kb, int KB, int gm,
+                                                int &ready_upto, volatile int *abort,
+                                                int *status) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        int v[8];
+        const int k0 = ready_upto + 1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = k0 + j < KB ? ld_relaxed_gpu(ctr + k0 + j) : 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (k0 + j >= KB || v[j] != gm || ready_upto != k0 + j - 1) break;
+            ready_upto = k0 + j;
+        }
+        if (ready_upto >= kb) {
+            __threadfence();  // acquire: the quantizer's stores happen-before what follows
+            return true;
+        }
+        if (it == 0) t0 = global_timer_ns();
+        if ((it & 15u) == 15u) {
+            if (*abort) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort = 1;
+                atomicExch(status, 6 /* FP8BQ_ERR_TIMEOUT */);
+                return false;
+            }
+        }
+    }
+}
 
 // Split-K tail: when the tiles leave a last wave of at most kTailMaxTiles tiles
 // on the persistent grid, each of those tiles is split K-wise into tail_parts
@@ -108,29 +197,57 @@ __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int
     tn = r / gm;
 }
 
+// Waits (bounded, like mbar_wait) until the upper 32 bits of the shared word
+// *p equal those of `tag`, and returns the word in `word`.
+__device__ __forceinline__ bool smem_tag_wait(volatile unsigned long long *p,
+                                              unsigned long long tag, unsigned long long &word,
+                                              volatile int *abort, int *status) {
+    word = *p;
+    if ((word >> 32) == (tag >> 32)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        word = *p;
+        if ((word >> 32) == (tag >> 32)) return true;
+        if ((it & 255u) == 0) {
+            if (*abort) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort = 1;
+                atomicExch(status, 6 /* FP8BQ_ERR_TIMEOUT */);
+                return false;
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
 // Promotes one K chunk of this thread's 128 TMEM columns into acc:
-// acc[i] = fma(P[i], scale, acc[i]).  The four 32-column TMEM loads are
-// software-pipelined (the next load is in flight while the FMAs of the
-// current one run); the last chunk is returned in `last` after its wait, so
-// the caller can release the TMEM buffer before finishing its FMAs.  Loads and
-// waits live in one asm statement so no register is read before its wait.
-__device__ __forceinline__ void promote_chunk(uint32_t taddr, float scale, float (&acc)[128],
-                                              float (&last)[32]) {
+// acc[i] = fma(P[i], scale, acc[i]), with the columns taken as two runs of 64:
+// acc[0..63] from TMEM columns taddr0 .. taddr0 + 63 with scale0, acc[64..127]
+// from taddr1 .. taddr1 + 63 with scale1 (for a plain tile, taddr1 = taddr0 +
+// 64 and scale1 = scale0).  The TMEM loads go in two batches of 64 columns,
+// one wait each: the second batch is in flight while the FMAs of the first
+// run, and it is returned in `last` after its wait, so the caller releases
+// the TMEM buffer after two load waits (not four) and finishes those 64 FMAs
+// afterwards (measured +3% on every prefill shape over four 32-column loads
+// with a wait each).  Loads and waits live in one asm statement so no
+// register is read before its wait.
+__device__ __forceinline__ void promote_chunk(uint32_t taddr0, uint32_t taddr1, float scale0,
+                                              float scale1, float (&acc)[128], float (&last)[64]) {
     asm volatile(
         "{\n\t"
         ".reg .f32 ra<32>, rb<32>;\n\t"
-        ".reg .b32 ta1, ta2, ta3;\n\t"
+        ".reg .b32 ta1, ta3;\n\t"
         "add.u32 ta1, %129, 32;\n\t"
-        "add.u32 ta2, %129, 64;\n\t"
-        "add.u32 ta3, %129, 96;\n\t"
+        "add.u32 ta3, %131, 32;\n\t"
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {ra0,ra1,ra2,ra3,ra4,ra5,ra6,ra7,ra8,ra9,ra10,ra11,ra12,ra13,ra14,ra15,ra16,ra17,ra18,ra19,ra20,ra21,ra22,ra23,ra24,ra25,ra26,ra27,ra28,ra29,ra30,ra31}, [%129];\n\t"
-        "tcgen05.wait::ld.sync.aligned;\n\t"
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {rb0,rb1,rb2,rb3,rb4,rb5,rb6,rb7,rb8,rb9,rb10,rb11,rb12,rb13,rb14,rb15,rb16,rb17,rb18,rb19,rb20,rb21,rb22,rb23,rb24,rb25,rb26,rb27,rb28,rb29,rb30,rb31}, [ta1];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%131];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [ta3];\n\t"
         "fma.rn.f32 %0, ra0, %128, %0;\n\t"
         "fma.rn.f32 %1, ra1, %128, %1;\n\t"
         "fma.rn.f32 %2, ra2, %128, %2;\n\t"
@@ -163,8 +280,6 @@ __device__ __forceinline__ void promote_chunk(uint32_t taddr, float scale, float
         "fma.rn.f32 %29, ra29, %128, %29;\n\t"
         "fma.rn.f32 %30, ra30, %128, %30;\n\t"
         "fma.rn.f32 %31, ra31, %128, %31;\n\t"
-        "tcgen05.wait::ld.sync.aligned;\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {ra0,ra1,ra2,ra3,ra4,ra5,ra6,ra7,ra8,ra9,ra10,ra11,ra12,ra13,ra14,ra15,ra16,ra17,ra18,ra19,ra20,ra21,ra22,ra23,ra24,ra25,ra26,ra27,ra28,ra29,ra30,ra31}, [ta2];\n\t"
         "fma.rn.f32 %32, rb0, %128, %32;\n\t"
         "fma.rn.f32 %33, rb1, %128, %33;\n\t"
         "fma.rn.f32 %34, rb2, %128, %34;\n\t"
@@ -198,74 +313,43 @@ __device__ __forceinline__ void promote_chunk(uint32_t taddr, float scale, float
         "fma.rn.f32 %62, rb30, %128, %62;\n\t"
         "fma.rn.f32 %63, rb31, %128, %63;\n\t"
         "tcgen05.wait::ld.sync.aligned;\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [ta3];\n\t"
-        "fma.rn.f32 %64, ra0, %128, %64;\n\t"
-        "fma.rn.f32 %65, ra1, %128, %65;\n\t"
-        "fma.rn.f32 %66, ra2, %128, %66;\n\t"
-        "fma.rn.f32 %67, ra3, %128, %67;\n\t"
-        "fma.rn.f32 %68, ra4, %128, %68;\n\t"
-        "fma.rn.f32 %69, ra5, %128, %69;\n\t"
-        "fma.rn.f32 %70, ra6, %128, %70;\n\t"
-        "fma.rn.f32 %71, ra7, %128, %71;\n\t"
-        "fma.rn.f32 %72, ra8, %128, %72;\n\t"
-        "fma.rn.f32 %73, ra9, %128, %73;\n\t"
-        "fma.rn.f32 %74, ra10, %128, %74;\n\t"
-        "fma.rn.f32 %75, ra11, %128, %75;\n\t"
-        "fma.rn.f32 %76, ra12, %128, %76;\n\t"
-        "fma.rn.f32 %77, ra13, %128, %77;\n\t"
-        "fma.rn.f32 %78, ra14, %128, %78;\n\t"
-        "fma.rn.f32 %79, ra15, %128, %79;\n\t"
-        "fma.rn.f32 %80, ra16, %128, %80;\n\t"
-        "fma.rn.f32 %81, ra17, %128, %81;\n\t"
-        "fma.rn.f32 %82, ra18, %128, %82;\n\t"
-        "fma.rn.f32 %83, ra19, %128, %83;\n\t"
-        "fma.rn.f32 %84, ra20, %128, %84;\n\t"
-        "fma.rn.f32 %85, ra21, %128, %85;\n\t"
-        "fma.rn.f32 %86, ra22, %128, %86;\n\t"
-        "fma.rn.f32 %87, ra23, %128, %87;\n\t"
-        "fma.rn.f32 %88, ra24, %128, %88;\n\t"
-        "fma.rn.f32 %89, ra25, %128, %89;\n\t"
-        "fma.rn.f32 %90, ra26, %128, %90;\n\t"
-        "fma.rn.f32 %91, ra27, %128, %91;\n\t"
-        "fma.rn.f32 %92, ra28, %128, %92;\n\t"
-        "fma.rn.f32 %93, ra29, %128, %93;\n\t"
-        "fma.rn.f32 %94, ra30, %128, %94;\n\t"
-        "fma.rn.f32 %95, ra31, %128, %95;\n\t"
-        "tcgen05.wait::ld.sync.aligned;\n\t"
         "}"
-        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+f"(acc[4]), "+f"(acc[5]),
-          "+f"(acc[6]), "+f"(acc[7]), "+f"(acc[8]), "+f"(acc[9]), "+f"(acc[10]), "+f"(acc[11]),
-          "+f"(acc[12]), "+f"(acc[13]), "+f"(acc[14]), "+f"(acc[15]), "+f"(acc[16]), "+f"(acc[17]),
-          "+f"(acc[18]), "+f"(acc[19]), "+f"(acc[20]), "+f"(acc[21]), "+f"(acc[22]), "+f"(acc[23]),
-          "+f"(acc[24]), "+f"(acc[25]), "+f"(acc[26]), "+f"(acc[27]), "+f"(acc[28]), "+f"(acc[29]),
-          "+f"(acc[30]), "+f"(acc[31]), "+f"(acc[32]), "+f"(acc[33]), "+f"(acc[34]), "+f"(acc[35]),
-          "+f"(acc[36]), "+f"(acc[37]), "+f"(acc[38]), "+f"(acc[39]), "+f"(acc[40]), "+f"(acc[41]),
-          "+f"(acc[42]), "+f"(acc[43]), "+f"(acc[44]), "+f"(acc[45]), "+f"(acc[46]), "+f"(acc[47]),
-          "+f"(acc[48]), "+f"(acc[49]), "+f"(acc[50]), "+f"(acc[51]), "+f"(acc[52]), "+f"(acc[53]),
-          "+f"(acc[54]), "+f"(acc[55]), "+f"(acc[56]), "+f"(acc[57]), "+f"(acc[58]), "+f"(acc[59]),
-          "+f"(acc[60]), "+f"(acc[61]), "+f"(acc[62]), "+f"(acc[63]), "+f"(acc[64]), "+f"(acc[65]),
-          "+f"(acc[66]), "+f"(acc[67]), "+f"(acc[68]), "+f"(acc[69]), "+f"(acc[70]), "+f"(acc[71]),
-          "+f"(acc[72]), "+f"(acc[73]), "+f"(acc[74]), "+f"(acc[75]), "+f"(acc[76]), "+f"(acc[77]),
-          "+f"(acc[78]), "+f"(acc[79]), "+f"(acc[80]), "+f"(acc[81]), "+f"(acc[82]), "+f"(acc[83]),
-          "+f"(acc[84]), "+f"(acc[85]), "+f"(acc[86]), "+f"(acc[87]), "+f"(acc[88]), "+f"(acc[89]),
-          "+f"(acc[90]), "+f"(acc[91]), "+f"(acc[92]), "+f"(acc[93]), "+f"(acc[94]), "+f"(acc[95]),
-          "=f"(last[0]), "=f"(last[1]), "=f"(last[2]), "=f"(last[3]), "=f"(last[4]), "=f"(last[5]),
-          "=f"(last[6]), "=f"(last[7]), "=f"(last[8]), "=f"(last[9]), "=f"(last[10]), "=f"(last[11]),
-          "=f"(last[12]), "=f"(last[13]), "=f"(last[14]), "=f"(last[15]), "=f"(last[16]),
-          "=f"(last[17]), "=f"(last[18]), "=f"(last[19]), "=f"(last[20]), "=f"(last[21]),
-          "=f"(last[22]), "=f"(last[23]), "=f"(last[24]), "=f"(last[25]), "=f"(last[26]),
-          "=f"(last[27]), "=f"(last[28]), "=f"(last[29]), "=f"(last[30]), "=f"(last[31])
-        : "f"(scale), "r"(taddr)
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+f"(acc[4]), "+f"(acc[5]), "+f"(acc[6]), "+f"(acc[7]), "+f"(acc[8]), "+f"(acc[9]), "+f"(acc[10]), "+f"(acc[11]), "+f"(acc[12]), "+f"(acc[13]), "+f"(acc[14]), "+f"(acc[15]), "+f"(acc[16]), "+f"(acc[17]), "+f"(acc[18]), "+f"(acc[19]), "+f"(acc[20]), "+f"(acc[21]), "+f"(acc[22]), "+f"(acc[23]), "+f"(acc[24]), "+f"(acc[25]), "+f"(acc[26]), "+f"(acc[27]), "+f"(acc[28]), "+f"(acc[29]), "+f"(acc[30]), "+f"(acc[31]), "+f"(acc[32]), "+f"(acc[33]), "+f"(acc[34]), "+f"(acc[35]), "+f"(acc[36]), "+f"(acc[37]), "+f"(acc[38]), "+f"(acc[39]), "+f"(acc[40]), "+f"(acc[41]), "+f"(acc[42]), "+f"(acc[43]), "+f"(acc[44]), "+f"(acc[45]), "+f"(acc[46]), "+f"(acc[47]), "+f"(acc[48]), "+f"(acc[49]), "+f"(acc[50]), "+f"(acc[51]), "+f"(acc[52]), "+f"(acc[53]), "+f"(acc[54]), "+f"(acc[55]), "+f"(acc[56]), "+f"(acc[57]), "+f"(acc[58]), "+f"(acc[59]), "+f"(acc[60]), "+f"(acc[61]), "+f"(acc[62]), "+f"(acc[63]), "=f"(last[0]), "=f"(last[1]), "=f"(last[2]), "=f"(last[3]), "=f"(last[4]), "=f"(last[5]), "=f"(last[6]), "=f"(last[7]), "=f"(last[8]), "=f"(last[9]), "=f"(last[10]), "=f"(last[11]), "=f"(last[12]), "=f"(last[13]), "=f"(last[14]), "=f"(last[15]), "=f"(last[16]), "=f"(last[17]), "=f"(last[18]), "=f"(last[19]), "=f"(last[20]), "=f"(last[21]), "=f"(last[22]), "=f"(last[23]), "=f"(last[24]), "=f"(last[25]), "=f"(last[26]), "=f"(last[27]), "=f"(last[28]), "=f"(last[29]), "=f"(last[30]), "=f"(last[31]), "=f"(last[32]), "=f"(last[33]), "=f"(last[34]), "=f"(last[35]), "=f"(last[36]), "=f"(last[37]), "=f"(last[38]), "=f"(last[39]), "=f"(last[40]), "=f"(last[41]), "=f"(last[42]), "=f"(last[43]), "=f"(last[44]), "=f"(last[45]), "=f"(last[46]), "=f"(last[47]), "=f"(last[48]), "=f"(last[49]), "=f"(last[50]), "=f"(last[51]), "=f"(last[52]), "=f"(last[53]), "=f"(last[54]), "=f"(last[55]), "=f"(last[56]), "=f"(last[57]), "=f"(last[58]), "=f"(last[59]), "=f"(last[60]), "=f"(last[61]), "=f"(last[62]), "=f"(last[63])
+        : "f"(scale0), "r"(taddr0), "f"(scale1), "r"(taddr1)
         : "memory");
 }
 
-template <int BN>
+// Outputs of the SiLU-gated epilogue (kSilu): for the fused gate/up weight
+// [2I, K] (gate rows [0, I), up rows [I, 2I)), tile column block tn holds gate
+// channels [128 tn, 128 tn + 128) in TMEM columns [0, 128) and the up channels
+// of the same indices in [128, 256); the tile's output is
+// h = BF16(silu(BF16 gate) * BF16 up) for those 128 channels, quantized as one
+// activation group: codes q [M, I], scales s [M, I/128], h [M, I] if h != null.
+struct SiluOut {
+    uint8_t *q;
+    float *s;
+    __nv_bfloat16 *h;
+};
+
+// kFusedAct (the linear layer): the A operand is quantized inside the launch.
+// Warp 3 of every CTA claims 128 x 128 chunks of the BF16 activation (tmap_x)
+// in the order the tiles consume them (m-tile group, then K chunk, then m-tile),
+// writes their E4M3 codes to fa.qa and their scales, transposed, to fa.saT, and
+// counts each finished chunk in its (group, K chunk) counter.  The producer
+// waits (bounded) for a chunk's counter before loading its codes, and a
+// 512-byte strip of its scales into a separate ring that the promotion warps
+// read.  No CTA waits for another CTA's progress except through those
+// counters, which any resident CTA's quantizer warp advances, so the grid need
+// not be co-resident.
+template <int BN, bool kSilu, bool kFusedAct>
 __global__ void __launch_bounds__(kNumThreads, 1)
 gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const float *__restrict__ sa,
                     const float *__restrict__ sw, __nv_bfloat16 *__restrict__ y, int M, int N,
-                    int K, int *status, int tail_parts, float *tail_partials, int *tail_counters) {
-    using L = Layout<BN>;
+                    int K, int *status, int tail_parts, float *tail_partials, int *tail_counters,
+                    SiluOut silu, const __grid_constant__ CUtensorMap tmap_x, FusedAct fa) {
+    static_assert(!(kSilu && kFusedAct), "one variant at a time");
+    using L = Layout<BN, kSilu, kFusedAct>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -274,13 +358,18 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     uint64_t *tfull = empty + kStages;
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;
+    uint64_t *sfull = drain + 1;       // kFusedAct: scale strips
+    uint64_t *sempty = sfull + kSaRing;
+    uint64_t *qfull = sempty + kSaRing;  // kFusedAct: quantizer input slots
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = K / BK;
     const int m_tiles = (M + BM - 1) / BM;
-    const int n_tiles = (N + BN - 1) / BN;
+    // kSilu: N = 2I weight rows, one tile per 128 output channels of h
+    const int I = N / 2;
+    const int n_tiles = kSilu ? I / 128 : (N + BN - 1) / BN;
     const int num_tiles = m_tiles * n_tiles;
     // with a split-K tail, the last wave's tiles are split into parts
     const int full_tiles =
@@ -297,12 +386,27 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&tempty[b], kPromoWarps);
         }
         mbar_init(drain, 2);
+        if constexpr (kFusedAct) {
+            for (int i = 0; i < kSaRing; ++i) {
+                mbar_init(&sfull[i], 1);
+                mbar_init(&sempty[i], kPromoWarps);
+            }
+            for (int i = 0; i < kQSlots; ++i) mbar_init(&qfull[i], 1);
+        }
         *abort_flag = 0;
         reinterpret_cast<uint32_t *>(smem + L::kMiscOff + 8)[0] = 0;  // tail verdict
         reinterpret_cast<uint32_t *>(smem + L::kMiscOff + 8)[1] = 0;  // tail arrivals
         fence_barrier_init();
+    }
+    if constexpr (kSilu) {
+        // no tile index matches this tag
+        unsigned long long *xchg = reinterpret_cast<unsigned long long *>(smem + L::kXchgOff);
+        for (int i = threadIdx.x; i < L::kXchgBytes / 8; i += kNumThreads) xchg[i] = ~0ull;
+    }
+    if (threadIdx.x == 0) {
         prefetch_tmap(&tmap_a);
         prefetch_tmap(&tmap_b);
+        if constexpr (kFusedAct) prefetch_tmap(&tmap_x);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, L::kTmemCols);
@@ -317,7 +421,8 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     grid_dependency_wait();
 
     if (warp < kFirstPromoWarp) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kFusedAct ? kProducerRegsFused
+                                                                            : kProducerRegs));
         if (warp == 0) {
             // ------------------------------------------------------------ TMA producer
             if (lane == 0) {
@@ -325,6 +430,8 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 int64_t issued = 0;
                 bool ok = true;
                 int t, kb0, kb1, part;
+                int cur_g = -1, ready_upto = -1;  // kFusedAct: chunks [0, ready_upto] of group cur_g are done
+                const uint64_t keep = l2_policy_evict_last();
                 for (int w = 0; ok && work_item(w, num_tiles, full_tiles, tail_parts, KB, t, kb0, kb1, part);
                      ++w) {
                     int tm, tn;
@@ -334,10 +441,45 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                             ok = false;
                             break;
                         }
+                        if constexpr (kFusedAct) {
+                            const int g = tm / kGroupM;
+                            if (g != cur_g) {
+                                cur_g = g;
+                                ready_upto = -1;
+                            }
+                            const int gm = min(kGroupM, m_tiles - g * kGroupM);
+                            if (kb > ready_upto) {
+                                if (!wait_act_chunks(fa.ctr + kActCtrBase + g * KB, kb, KB, gm,
+                                                     ready_upto, abort_flag, status)) {
+                                    ok = false;
+                                    break;
+                                }
+                                // once per newly acquired batch of chunks: the
+                                // TMA loads below read what the acquire made visible
+                                fence_proxy_async_global();
+                            }
+                            const uint32_t si = static_cast<uint32_t>(issued % kSaRing);
+                            const uint32_t sp = static_cast<uint32_t>((issued / kSaRing) & 1);
+                            if (!mbar_wait(&sempty[si], sp ^ 1, abort_flag, status)) {
+                                ok = false;
+                                break;
+                            }
+                            mbar_arrive_expect_tx(&sfull[si], kSaStrip);
+                            bulk_load(smem + L::kSaOff + si * kSaStrip,
+                                      fa.saT + static_cast<int64_t>(kb) * fa.m_pad + tm * BM, kSaStrip,
+                                      &sfull[si], keep);
+                        }
                         uint8_t *st = smem + stage * L::kStage;
                         mbar_arrive_expect_tx(&full[stage], L::kStage);
                         tma_load_2d(st, &tmap_a, &full[stage], kb * BK, tm * BM);
-                        tma_load_2d(st + L::kA, &tmap_b, &full[stage], kb * BK, tn * BN);
+                        if constexpr (kSilu) {
+                            // gate block tn above up block tn (128-row boxes)
+                            tma_load_2d(st + L::kA, &tmap_b, &full[stage], kb * BK, tn * 128);
+                            tma_load_2d(st + L::kA + 128 * BK, &tmap_b, &full[stage], kb * BK,
+                                        I + tn * 128);
+                        } else {
+                            tma_load_2d(st + L::kA, &tmap_b, &full[stage], kb * BK, tn * BN);
+                        }
                         ++issued;
                         if (++stage == kStages) {
                             stage = 0;
@@ -349,6 +491,109 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 for (int64_t i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
                     mbar_wait(&full[i % kStages], static_cast<uint32_t>((i / kStages) & 1), nullptr,
                               status);
+                if constexpr (kFusedAct)
+                    for (int64_t i = (issued > kSaRing ? issued - kSaRing : 0); i < issued; ++i)
+                        mbar_wait(&sfull[i % kSaRing], static_cast<uint32_t>((i / kSaRing) & 1),
+                                  nullptr, status);
+            }
+        } else if (kFusedAct && warp == 3) {
+            // ------------------------------------------------------------ activation quantizer
+            // Chunk c -> (m-tile group g, K chunk kb, m-tile tm), in the order the
+            // tiles consume them.  Two input slots: the next chunk's load is in
+            // flight while this one is encoded.  A slot holds the chunk's two
+            // 64-channel halves, [128 rows][128 B] each in the 128-byte swizzle
+            // (16-byte unit j of row r at r*128 + 16*(j ^ (r & 7))), so a lane
+            // can own a whole row: lane l encodes rows l, l+32, l+64, l+96, with
+            // no shuffles, and conflict-free shared-memory accesses.  The codes
+            // overwrite the first half in place (a row's unit is read before it
+            // is written) in the same swizzled layout, which one TMA store
+            // writes to the code matrix through the A operand's tensor map.
+            const int64_t n_chunks = static_cast<int64_t>(m_tiles) * KB;
+            const uint64_t stream_once = l2_policy_evict_first();
+            auto claim = [&]() -> int64_t {
+                int c = 0;
+                if (lane == 0) c = atomicAdd(fa.ctr + kActClaimSlot, 1);
+                return __shfl_sync(0xFFFFFFFFu, c, 0);
+            };
+            auto coords = [&](int64_t c, int &g, int &kb, int &tm) {
+                g = static_cast<int>(c / (static_cast<int64_t>(KB) * kGroupM));
+                const int64_t r = c - static_cast<int64_t>(g) * KB * kGroupM;
+                const int gm = min(kGroupM, m_tiles - g * kGroupM);
+                kb = static_cast<int>(r / gm);
+                tm = g * kGroupM + static_cast<int>(r % gm);
+            };
+            auto issue = [&](int64_t c, uint32_t slot) {
+                __syncwarp();  // every lane's reads of the slot come before the load
+                if (lane == 0) {
+                    int g, kb, tm;
+                    coords(c, g, kb, tm);
+                    uint8_t *dst = smem + L::kQOff + slot * kQChunkBytes;
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(&qfull[slot], kQChunkBytes);
+                    tma_load_2d_hint(dst, &tmap_x, &qfull[slot], kb * BK, tm * BM, stream_once);
+                    tma_load_2d_hint(dst + kQChunkBytes / 2, &tmap_x, &qfull[slot], kb * BK + BK / 2,
+                                     tm * BM, stream_once);
+                }
+            };
+            uint32_t slot = 0, qphase[kQSlots] = {0, 0};
+            int64_t cur = claim();
+            if (cur < n_chunks) issue(cur, 0);
+            while (cur < n_chunks) {
+                const int64_t nxt = claim();
+                if (nxt < n_chunks) issue(nxt, slot ^ 1);
+                bool okw = mbar_wait(&qfull[slot], qphase[slot], abort_flag, status);
+                if (!__all_sync(0xFFFFFFFFu, okw)) {
+                    if (nxt < n_chunks)  // let the load in flight land before the CTA exits
+                        mbar_wait(&qfull[slot ^ 1], qphase[slot ^ 1], nullptr, status);
+                    break;
+                }
+                qphase[slot] ^= 1;
+                int g, kb, tm;
+                coords(cur, g, kb, tm);
+                uint8_t *h0 = smem + L::kQOff + slot * kQChunkBytes;
+                const uint8_t *h1 = h0 + kQChunkBytes / 2;
+                float *st = fa.saT + static_cast<int64_t>(kb) * fa.m_pad + tm * BM;
+                for (int rb = 0; rb < BM / 32; ++rb) {
+                    const int r = rb * 32 + lane;
+                    const int x7 = r & 7;
+                    uint8_t *r0 = h0 + r * 128;
+                    const uint8_t *r1 = h1 + r * 128;
+                    uint32_t m = 0;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        m = max(m, amax_bits8(*reinterpret_cast<const uint4 *>(r0 + ((u ^ x7) << 4))));
+                        m = max(m, amax_bits8(*reinterpret_cast<const uint4 *>(r1 + ((u ^ x7) << 4))));
+                    }
+                    const float scale = scale_from_amax_bits(m);
+                    const float yr = __frcp_rn(scale);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        // channels 16v .. 16v + 15: units 2v, 2v + 1 of the row
+                        const uint8_t *rs = v < 4 ? r0 : r1;
+                        const int ua = (2 * v) & 7;
+                        const uint4 a = *reinterpret_cast<const uint4 *>(rs + ((ua ^ x7) << 4));
+                        const uint4 b = *reinterpret_cast<const uint4 *>(rs + (((ua + 1) ^ x7) << 4));
+                        const uint2 ca = encode8_y(a, scale, yr);
+                        const uint2 cb = encode8_y(b, scale, yr);
+                        *reinterpret_cast<uint4 *>(r0 + ((v ^ x7) << 4)) = make_uint4(ca.x, ca.y, cb.x, cb.y);
+                    }
+                    st[r] = scale;  // rows past M: scale 1 (zero-filled input)
+                }
+                // The code tile (rows past M are not stored), then the chunk's
+                // counter: the store's writes are complete and ordered before
+                // the release, and before other CTAs' TMA loads of them.
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmap_a, h0, kb * BK, tm * BM);
+                    bulk_commit_group();
+                    bulk_wait_group_all();
+                    fence_proxy_async_global();
+                    __threadfence();
+                    atomicAdd(fa.ctr + kActCtrBase + g * KB + kb, 1);
+                }
+                cur = nxt;
+                slot ^= 1;
             }
         } else if (warp == 1 || warp == 2) {
             // ------------------------------------------------------------ MMA issuers
@@ -390,7 +635,8 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             }
         }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kFusedAct ? kConsumerRegsFused
+                                                                            : kConsumerRegs));
         // ------------------------------------------------------------ promotion + epilogue
         const int pw = warp - kFirstPromoWarp;
         const int quarter = warp & 3;  // TMEM lane quarter accessible to this warp
@@ -401,6 +647,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
         volatile uint32_t *tail_last = reinterpret_cast<volatile uint32_t *>(smem + L::kMiscOff + 8);
         uint32_t *tail_arrived = reinterpret_cast<uint32_t *>(smem + L::kMiscOff + 12);
         uint32_t buf = 0, bphase = 0;
+        int64_t ci = 0;  // kFusedAct: chunk index over the CTA's work, as the producer counts it
         bool ok = true;
         int t, kb0, kb1, part;
         for (int w = 0; ok && work_item(w, num_tiles, full_tiles, tail_parts, KB, t, kb0, kb1, part);
@@ -408,53 +655,142 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             int tm, tn;
             tile_coords(t, m_tiles, n_tiles, tm, tn);
             const int grow = tm * BM + row_in_tile;
-            const int gcol = tn * BN + half * 128;
+            // plain: this thread's 128 output columns, one weight block; SiLU:
+            // 64 gate and the same 64 up channels, two weight blocks
+            const int gcol = kSilu ? tn * 128 + half * 64 : tn * BN + half * 128;
             const bool row_ok = grow < M;
             const bool col_ok = gcol < N;
             const float *sa_row = sa + static_cast<int64_t>(row_ok ? grow : 0) * KB;
-            const float *sw_row = sw + static_cast<int64_t>(col_ok ? gcol / 128 : 0) * KB;
+            const float *sw_row =
+                sw + static_cast<int64_t>(kSilu ? tn : (col_ok ? gcol / 128 : 0)) * KB;
+            const float *swu_row = sw + static_cast<int64_t>(I / 128 + tn) * KB;  // kSilu: up block
 
             float acc[128];
 #pragma unroll
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
             // scales of the next kScaleLookahead chunks, in a register ring
-            float sa_q[kScaleLookahead], sw_q[kScaleLookahead];
+            float sa_q[kScaleLookahead], sw_q[kScaleLookahead], swu_q[kScaleLookahead];
 #pragma unroll
             for (int j = 0; j < kScaleLookahead; ++j) {
-                sa_q[j] = (row_ok && kb0 + j < kb1) ? __ldg(sa_row + kb0 + j) : 0.0f;
+                sa_q[j] = (!kFusedAct && row_ok && kb0 + j < kb1) ? __ldg(sa_row + kb0 + j) : 0.0f;
                 sw_q[j] = (col_ok && kb0 + j < kb1) ? __ldg(sw_row + kb0 + j) : 0.0f;
+                if constexpr (kSilu) swu_q[j] = kb0 + j < kb1 ? __ldg(swu_row + kb0 + j) : 0.0f;
             }
             for (int kbb = kb0; kbb < kb1 && ok; kbb += kScaleLookahead) {
 #pragma unroll
                 for (int j = 0; j < kScaleLookahead; ++j) {
                     const int kb = kbb + j;
                     if (kb >= kb1) break;
-                    const float scale = sa_q[j] * sw_q[j];
+                    float sa_v = sa_q[j];
+                    if constexpr (kFusedAct) {
+                        // this chunk's activation scales, from the strip ring
+                        const uint32_t si = static_cast<uint32_t>(ci % kSaRing);
+                        if (!mbar_wait(&sfull[si], static_cast<uint32_t>((ci / kSaRing) & 1), abort_flag,
+                                       status)) {
+                            ok = false;
+                            break;
+                        }
+                        sa_v = reinterpret_cast<const float *>(smem + L::kSaOff + si * kSaStrip)[row_in_tile];
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sempty[si]);
+                        ++ci;
+                    }
+                    const float scale = sa_v * sw_q[j];
+                    const float scale1 = kSilu ? sa_v * swu_q[j] : scale;
                     const int kn = kb + kScaleLookahead;
                     if (kn < kb1) {
-                        sa_q[j] = row_ok ? __ldg(sa_row + kn) : 0.0f;
+                        sa_q[j] = (!kFusedAct && row_ok) ? __ldg(sa_row + kn) : 0.0f;
                         sw_q[j] = col_ok ? __ldg(sw_row + kn) : 0.0f;
+                        if constexpr (kSilu) swu_q[j] = __ldg(swu_row + kn);
                     }
                     if (!mbar_wait(&tfull[buf], bphase, abort_flag, status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t taddr = tmem_base +
-                                           (static_cast<uint32_t>(quarter * 32) << 16) +
-                                           buf * BN + half * 128;
-                    float last[32];
-                    promote_chunk(taddr, scale, acc, last);
+                    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                           buf * BN;
+                    const uint32_t taddr0 = tbase + (kSilu ? half * 64 : half * 128);
+                    const uint32_t taddr1 = kSilu ? tbase + 128 + half * 64 : taddr0 + 64;
+                    float last[64];
+                    promote_chunk(taddr0, taddr1, scale, scale1, acc, last);
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&tempty[buf]);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(last[i], scale, acc[96 + i]);
+                    for (int i = 0; i < 64; ++i) acc[64 + i] = fmaf(last[i], scale1, acc[64 + i]);
                     buf ^= 1;
                     if (buf == 0) bphase ^= 1;
                 }
             }
             if (!ok) break;
+            if constexpr (kSilu) {
+                // h = BF16(silu(g) * u) with g, u the BF16-rounded accumulators
+                // (what the plain GEMM would store), by the standalone SiLU
+                // kernel's arithmetic; then one activation group of 128
+                // channels per row, split over the two column halves, whose
+                // maxima meet in shared memory.
+                uint32_t hb[32];
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const uint4 gv = make_uint4(pack_bf16x2(acc[8 * v + 0], acc[8 * v + 1]),
+                                                pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
+                                                pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]),
+                                                pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+                    const uint4 uv = make_uint4(pack_bf16x2(acc[64 + 8 * v + 0], acc[64 + 8 * v + 1]),
+                                                pack_bf16x2(acc[64 + 8 * v + 2], acc[64 + 8 * v + 3]),
+                                                pack_bf16x2(acc[64 + 8 * v + 4], acc[64 + 8 * v + 5]),
+                                                pack_bf16x2(acc[64 + 8 * v + 6], acc[64 + 8 * v + 7]));
+                    const uint4 h8 = silu_mul8(gv, uv);
+                    hb[4 * v + 0] = h8.x;
+                    hb[4 * v + 1] = h8.y;
+                    hb[4 * v + 2] = h8.z;
+                    hb[4 * v + 3] = h8.w;
+                }
+                uint32_t amax = 0;
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    amax = max(amax, amax_bits8(make_uint4(hb[4 * v], hb[4 * v + 1], hb[4 * v + 2],
+                                                           hb[4 * v + 3])));
+                // The partner thread (same row, other half) is in the other
+                // promotion warpgroup.  Each publishes (tile index, amax) in one
+                // 64-bit word and waits, bounded, for the partner's word of this
+                // tile; slots alternate by tile parity, so a slot is rewritten
+                // only after the partner has read it.
+                volatile unsigned long long *xchg =
+                    reinterpret_cast<volatile unsigned long long *>(smem + L::kXchgOff) +
+                    (w & 1) * (2 * BM);
+                const unsigned long long tag = static_cast<unsigned long long>(w) << 32;
+                xchg[row_in_tile * 2 + half] = tag | amax;
+                unsigned long long other;
+                if (!smem_tag_wait(&xchg[row_in_tile * 2 + (half ^ 1)], tag, other, abort_flag,
+                                   status)) {
+                    ok = false;
+                    break;
+                }
+                amax = max(amax, static_cast<uint32_t>(other));
+                const float scale = scale_from_amax_bits(amax);
+                if (row_ok) {
+                    const int64_t c0 = static_cast<int64_t>(grow) * I + tn * 128 + half * 64;
+                    uint4 *qd = reinterpret_cast<uint4 *>(silu.q + c0);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const uint2 lo = encode8(make_uint4(hb[8 * v], hb[8 * v + 1], hb[8 * v + 2],
+                                                            hb[8 * v + 3]), scale);
+                        const uint2 hi = encode8(make_uint4(hb[8 * v + 4], hb[8 * v + 5],
+                                                            hb[8 * v + 6], hb[8 * v + 7]), scale);
+                        qd[v] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+                    }
+                    if (half == 0) silu.s[static_cast<int64_t>(grow) * (I / 128) + tn] = scale;
+                    if (silu.h != nullptr) {
+                        uint4 *hd = reinterpret_cast<uint4 *>(silu.h + c0);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            hd[v] = make_uint4(hb[4 * v], hb[4 * v + 1], hb[4 * v + 2], hb[4 * v + 3]);
+                    }
+                }
+                continue;
+            }
             const bool write = part < 0;  // full tile: write its output from registers
             if (part >= 0) {
                 // Tail part: publish the FP32 partial [128 rows][256 cols] of
@@ -528,6 +864,26 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, L::kTmemCols);
+    }
+    if constexpr (kFusedAct) {
+        // The last CTA to get here zeroes the quantization counters (every
+        // other CTA, its quantizer warp included, has finished with them), so
+        // the workspace header is back in its initial state for the next call.
+        volatile int *last = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 16);
+        if (threadIdx.x == 0) {
+            __threadfence();
+            *last = atomicAdd(fa.ctr + kActExitSlot, 1) == static_cast<int>(gridDim.x) - 1;
+        }
+        __syncthreads();
+        if (*last) {
+            __threadfence();
+            const int n = KB * ((m_tiles + kGroupM - 1) / kGroupM);
+            for (int i = threadIdx.x; i < n; i += kNumThreads) fa.ctr[kActCtrBase + i] = 0;
+            if (threadIdx.x == 0) {
+                fa.ctr[kActClaimSlot] = 0;
+                fa.ctr[kActExitSlot] = 0;
+            }
+        }
     }
 }
 

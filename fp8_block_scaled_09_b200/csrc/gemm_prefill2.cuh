@@ -243,8 +243,8 @@ gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const uint32_t taddr = tmem_base +
                                            (static_cast<uint32_t>(quarter * 32) << 16) +
                                            buf * BN + half * 128;
-                    float last[32];
-                    promote_chunk(taddr, scale, acc, last);
+                    float last[64];
+                    promote_chunk(taddr, taddr + 64, scale, scale, acc, last);
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) {
@@ -254,7 +254,7 @@ gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                             mbar_arrive_remote_relaxed(buf ? tempty0_b1 : tempty0_b0);
                     }
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(last[i], scale, acc[96 + i]);
+                    for (int i = 0; i < 64; ++i) acc[64 + i] = fmaf(last[i], scale, acc[64 + i]);
                     buf ^= 1;
                     if (buf == 0) bphase ^= 1;
                 }

@@ -57,6 +57,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
+// try_wait whose thread may stay suspended up to hint_ns while the phase is
+// incomplete (it resumes as soon as the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
 // try_wait that acquires at cluster scope: for barriers that other CTAs of the
 // cluster arrive on.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
@@ -75,11 +90,17 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 // (returns false) when *abort (if not null) is set by another thread of the
 // CTA, or after kWaitLimitNs, in which case it sets *abort and stores
 // FP8BQ_ERR_TIMEOUT in the device status word *status (global memory).
-template <bool kClusterScope = false>
+// kSuspendNs > 0: each test may keep the waiting thread suspended up to that
+// long (it resumes when the phase completes), so waiting warps take fewer
+// issue slots (measured -2% per decode GEMM launch with 10 us; the prefill
+// GEMM was slightly slower with it, so it keeps plain tests).
+template <bool kClusterScope = false, uint32_t kSuspendNs = 0>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           int *status, uint64_t limit_ns = kWaitLimitNs) {
     auto ready = [&]() {
-        return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+        if constexpr (kClusterScope) return mbar_try_wait_cluster(bar, parity);
+        if constexpr (kSuspendNs > 0) return mbar_try_wait_hint(bar, parity, kSuspendNs);
+        return mbar_try_wait(bar, parity);
     };
     if (ready()) return true;
     const uint64_t t0 = global_timer_ns();
@@ -143,6 +164,29 @@ __device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *m
         ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "l"(policy)
         : "memory");
+}
+
+// 2-D tile store shared -> global (the map's box and swizzle describe the
+// shared-memory tile), tracked as a bulk async-group of this thread.  Out-of-
+// bounds parts of the box are not written.  x, y >= 0.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x,
+                                             int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_addr(src)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Closes this thread's current bulk async-group.
+__device__ __forceinline__ void bulk_commit_group() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until all of this thread's bulk async-groups are complete (their
+// writes to global memory performed).
+__device__ __forceinline__ void bulk_wait_group_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Untiled bulk copy global -> shared: both addresses 16-byte aligned, `bytes` a

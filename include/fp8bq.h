@@ -81,7 +81,7 @@ typedef enum {
 } fp8bq_status;
 
 /* Operation selector for fp8bq_workspace_size. */
-typedef enum { FP8BQ_OP_GEMM = 0, FP8BQ_OP_LINEAR = 1 } fp8bq_op;
+typedef enum { FP8BQ_OP_GEMM = 0, FP8BQ_OP_LINEAR = 1, FP8BQ_OP_GEMM_SILU = 2 } fp8bq_op;
 
 /*
  * Dynamic per-token, group-128 activation quantization (page
@@ -123,6 +123,13 @@ FP8BQ_API fp8bq_status fp8bq_quantize_weight(const void *w_bf16, int64_t N, int6
  *       state); calls that share a workspace must be ordered (same stream).
  * Output accuracy: |y - ref| <= 1e-2 |ref| + 2e-3 rms(ref) against the FP64 sum
  * of the dequantized operands; results are deterministic for a given shape.
+ * For M <= 16 the call starts reading qw / sw while the previous kernel in the
+ * stream may still be running, and lets the next kernel start while its own
+ * last blocks finish (programmatic dependent launch), so consecutive calls
+ * overlap.  qa, sa and the workspace are read only after the previous kernel
+ * has completed.  Reading qw / sw early is safe after this library's weight
+ * quantizers, which never let a successor start early; qw / sw must not be
+ * written by a foreign kernel that does.
  */
 FP8BQ_API fp8bq_status fp8bq_gemm(const uint8_t *qa, const float *sa, const uint8_t *qw, const float *sw,
                         int64_t M, int64_t N, int64_t K, void *y_bf16, void *workspace,
@@ -190,6 +197,35 @@ FP8BQ_API fp8bq_status fp8bq_silu_mul_quantize(const void *gu_bf16, int64_t M, i
                                                void *stream);
 
 /*
+ * Gate/up projection of the MLP with the SiLU-gated product quantized for the
+ * down projection in the same pass (pages "ProCreations/Nanbeige4.3-33B-DFlash2",
+ * "Architecture and checkpoint format": separate gate and up projections of the
+ * MLP; "ProCreations/Nanbeige4.3-33B-FP8", introduction: every linear layer,
+ * the down projection included, takes group-128 dynamically quantized
+ * activations).  With gu = gemm(qa, sa, qw, sw) the BF16 [M, 2I] output of the
+ * fused gate/up weight, this computes exactly
+ *     fp8bq_silu_mul_quantize(gu, M, I, q_e4m3, s, h_bf16)
+ * (same codes, scales and h, bit for bit) without gu ever reaching memory for
+ * M > 128: there the GEMM's epilogue holds 128 gate channels and the same 128
+ * up channels of a row and writes their h codes and scale directly.
+ *   qa, sa : in, activation codes [M, K] and scales [M, K/128]
+ *   qw, sw : in, the fused gate/up weight: codes [2I, K] (gate rows [0, I), up
+ *            rows [I, 2I)) and scales [2I/128, K/128], e.g. from
+ *            fp8bq_quantize_weight of the BF16 [2I, K] weight
+ *   q_e4m3, s : out, the down projection's input codes [M, I], scales [M, I/128]
+ *   h_bf16 : out, optional BF16 h [M, I] (NULL: not stored)
+ *   workspace : at least fp8bq_workspace_size(FP8BQ_OP_GEMM_SILU, M, 2I, K)
+ *       bytes (0 for M > 128; for M <= 128 the call runs the decode GEMM into
+ *       the workspace and then the SiLU kernel), same state rule as fp8bq_gemm.
+ * I a multiple of 128, K a multiple of 128; pointers 16-byte aligned.
+ */
+FP8BQ_API fp8bq_status fp8bq_gemm_silu_mul_quantize(const uint8_t *qa, const float *sa,
+                                                    const uint8_t *qw, const float *sw, int64_t M,
+                                                    int64_t I, int64_t K, uint8_t *q_e4m3,
+                                                    float *s, void *h_bf16, void *workspace,
+                                                    size_t ws_bytes, void *stream);
+
+/*
  * NVFP4 weight-only format with BF16 activations (page
  * "ProCreations/Nanbeige4.3-33B-NVFP4-A16", recipe paragraph: FP4 E2M1 weights
  * in groups of 16 with E4M3 block scales and a global weight scale; activations
@@ -254,11 +290,14 @@ FP8BQ_API fp8bq_status fp8bq_gemm_noalloc(const uint8_t *qa, const float *sa, co
  * a fixed order, so results stay deterministic and within the same
  * tolerance), which a smaller workspace goes without.  The fused linear
  * requires, besides the GEMM's part (never less than its 16 KB counter
- * header), its activation codes and scales.
+ * header), its activation codes and scales.  FP8BQ_OP_GEMM_SILU takes N = 2I
+ * (the fused gate/up weight's rows): 0 for M > 128, else the GEMM's part (at
+ * least the header) and the BF16 gate/up output [M, 2I].
  * Every workspace starts with the same 16 KB header of split-K counters, at
- * offset 0 for both operations and every shape, and every successful call
- * leaves them at zero: one workspace, large enough for each call, can serve
- * any sequence of fp8bq_gemm and fp8bq_linear calls in stream order. */
+ * offset 0 for every operation and shape, and every successful call leaves
+ * them at zero: one workspace, large enough for each call, can serve any
+ * sequence of fp8bq_gemm, fp8bq_linear and fp8bq_gemm_silu_mul_quantize calls
+ * in stream order. */
 FP8BQ_API size_t fp8bq_workspace_size(int op, int64_t M, int64_t N, int64_t K);
 
 /* Put a workspace into its initial state (zero-fills ws_bytes bytes on the

@@ -41,7 +41,7 @@ def test_header_declares_the_abi():
     names = declared_functions()
     for n in ("fp8bq_quantize_act", "fp8bq_quantize_weight", "fp8bq_gemm", "fp8bq_linear",
               "fp8bq_workspace_size", "fp8bq_last_device_status", "fp8bq_status_string",
-              "fp8bq_kv_write_e4m3", "fp8bq_silu_mul_quantize"):
+              "fp8bq_kv_write_e4m3", "fp8bq_silu_mul_quantize", "fp8bq_gemm_silu_mul_quantize"):
         assert n in names
 
 
@@ -122,15 +122,15 @@ def test_linear_argument_errors(L):
     assert f(GOOD, GOOD, None, 300, 256, 256, GOOD, GOOD, ws, None) == INVALID
     assert f(ODD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws, None) == MISALIGNED
     # for M > 128: the 16 KB counter header (kept at offset 0 of every
-    # workspace), then the activation codes and scales, all required (at this K
-    # the prefill GEMM has no split-K tail to report)
+    # workspace), then the activation codes and scales (transposed, rows padded
+    # to 384), all required (at this K the prefill GEMM has no split-K tail)
     up = lambda b: -(-b // 256) * 256                # each part padded to 256 bytes
-    assert ws == 16384 + up(300 * 256) + up(300 * 2 * 4)
+    assert ws == 16384 + up(300 * 256) + up(384 * 2 * 4)
     assert f(GOOD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws - 256, None) == WORKSPACE
     # at K >= 16384 the optional tail (header included) replaces the bare header
     ws_long = fp8bq.workspace_size(fp8bq.OP_LINEAR, 300, 256, 16384)
     tail = 16384 + 16 * 4 * 128 * 256 * 4
-    assert ws_long == tail + up(300 * 16384) + up(300 * 128 * 4)
+    assert ws_long == tail + up(300 * 16384) + up(384 * 128 * 4)
     assert f(GOOD, GOOD, GOOD, 300, 256, 16384, GOOD, GOOD, ws_long - tail + 16384 - 256,
              None) == WORKSPACE
     assert f(None, None, None, 0, 256, 256, None, None, 0, None) == OK
@@ -161,6 +161,22 @@ def test_silu_mul_quantize_argument_errors(L):
     assert f(GOOD, 4, 128, GOOD, None, None, None) == INVALID
     assert f(GOOD, 4, 128, ODD, GOOD, None, None) == MISALIGNED
     assert f(GOOD, 4, 128, GOOD, GOOD, ODD, None) == MISALIGNED  # optional h, if given
+
+
+def test_gemm_silu_mul_quantize_argument_errors(L):
+    f = L.fp8bq_gemm_silu_mul_quantize
+    #        qa    sa    qw    sw    M    I    K    q     s     h     ws    bytes
+    assert f(GOOD, GOOD, GOOD, GOOD, 300, 100, 256, GOOD, GOOD, None, None, 0, None) == SHAPE
+    assert f(GOOD, GOOD, GOOD, GOOD, 300, 128, 200, GOOD, GOOD, None, None, 0, None) == SHAPE
+    assert f(GOOD, GOOD, GOOD, GOOD, -1, 128, 256, GOOD, GOOD, None, None, 0, None) == SHAPE
+    assert f(None, None, None, None, 0, 128, 256, None, None, None, None, 0, None) == OK
+    assert f(GOOD, GOOD, GOOD, GOOD, 300, 128, 256, None, GOOD, None, None, 0, None) == INVALID
+    assert f(GOOD, GOOD, GOOD, GOOD, 300, 128, 256, GOOD, GOOD, ODD, None, 0, None) == MISALIGNED
+    # decode-sized M needs its workspace (GEMM part + BF16 gate/up output)
+    assert f(GOOD, GOOD, GOOD, GOOD, 8, 128, 256, GOOD, GOOD, None, None, 0, None) == WORKSPACE
+    need = fp8bq.workspace_size(fp8bq.OP_GEMM_SILU, 8, 256, 256)
+    assert f(GOOD, GOOD, GOOD, GOOD, 8, 128, 256, GOOD, GOOD, None, GOOD, need - 256,
+             None) == WORKSPACE
 
 
 def test_nvfp4_argument_errors(L):
@@ -205,8 +221,17 @@ def test_workspace_sizes(L):
     assert lin(8192, 9216, 7168) == 16384 + 8192 * 7168 + 8192 * 56 * 4
     assert lin(16, 9216, 7168) == d + 16 * 7168 + up(16 * 56 * 4)
     assert lin(4096, 7168, 21504) == tail + 4096 * 21504 + 4096 * 168 * 4
+    # M > 128: the scales are kept transposed, [K/128, M rounded up to 128]
+    assert lin(300, 256, 1024) == 16384 + up(300 * 1024) + up(384 * 8 * 4)
     for args in ((1, 128, 128), (17, 384, 1024), (4096, 7168, 21504)):
         assert lin(*args) % 256 == 0 and g(*args) % 256 == 0
+    # gate/up with the SiLU epilogue (N = 2I): nothing on the fused prefill path;
+    # for M <= 128 the GEMM's part (at least the header) and the BF16 gate/up output
+    gs = lambda M, N, K: fp8bq.workspace_size(fp8bq.OP_GEMM_SILU, M, N, K)
+    assert gs(129, 16384, 7168) == 0 and gs(4096, 16384, 7168) == 0
+    assert gs(8, 16384, 7168) == g(8, 16384, 7168) + 8 * 16384 * 2
+    assert gs(1, 256, 128) == max(g(1, 256, 128), 16384) + up(256 * 2)
+    assert gs(8, 384, 7168) == 0                                   # N = 2I needs I % 128 == 0
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="valid calls would launch kernels on fake pointers")
@@ -216,6 +241,8 @@ def test_valid_call_without_device_reports_no_device(L):
     assert L.fp8bq_selftest_timeout(20000, None) == NODEV
     assert L.fp8bq_kv_write_e4m3(GOOD, GOOD, 1024, 4, 1024, GOOD, GOOD, GOOD, 8, 1024, None) == NODEV
     assert L.fp8bq_silu_mul_quantize(GOOD, 4, 128, GOOD, GOOD, None, None) == NODEV
+    assert L.fp8bq_gemm_silu_mul_quantize(GOOD, GOOD, GOOD, GOOD, 300, 128, 256, GOOD, GOOD, None,
+                                          None, 0, None) == NODEV
     assert L.fp8bq_nvfp4_quantize_weight(GOOD, 128, 256, GOOD, GOOD, GOOD, None) == NODEV
     assert L.fp8bq_nvfp4_gemm_a16(GOOD, GOOD, GOOD, GOOD, 4, 128, 256, GOOD, None) == NODEV
 

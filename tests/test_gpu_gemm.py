@@ -177,7 +177,8 @@ def test_gemm_empty_m_is_noop():
 LINEAR_SHAPES = [(1, 1024, 7168), (16, 1024, 7168), (5, 384, 640), (1, 9216, 7168),
                  (8, 7168, 7168), (17, 1152, 512), (32, 2048, 2048), (31, 640, 7168),
                  (4, 19200, 512), (3, 32768, 256), (12, 16384, 1024), (20, 256, 128000),
-                 (33, 256, 1024), (128, 1152, 7168), (192, 640, 2048), (700, 384, 7168)]
+                 (33, 256, 1024), (128, 1152, 7168), (192, 640, 2048), (700, 384, 7168),
+                 (129, 256, 128), (2100, 512, 1024), (4096, 256, 384)]
 
 
 @pytest.mark.parametrize("M,N,K", LINEAR_SHAPES)
@@ -195,12 +196,21 @@ def test_linear_matches_oracle_and_unfused_path(M, N, K):
     y2 = fp8bq.gemm(gq, gs, to_dev_codes(qw), to_dev_f32(sw))
     assert torch.equal(y.t.view(torch.int16), y2.view(torch.int16))
     # the linear's scratch (behind the GEMM's part of a workspace of the
-    # reported size) holds exactly those codes and scales
+    # reported size) holds exactly those codes and scales; for M > 128 (one
+    # launch: quantized inside the GEMM) the scales are stored transposed,
+    # [K/128, M rounded up to 128]
     up = lambda b: -(-b // 256) * 256
-    off = ws.numel() - up(M * K) - up(M * (K // 128) * 4)
+    rows_s = M if M <= 128 else -(-M // 128) * 128
+    off = ws.numel() - up(M * K) - up(rows_s * (K // 128) * 4)
     assert torch.equal(ws[off:off + M * K].view(M, K), gq)
     so = off + up(M * K)
-    assert torch.equal(ws[so:so + M * (K // 128) * 4].view(torch.float32).view(M, K // 128), gs)
+    scales = ws[so:so + rows_s * (K // 128) * 4].view(torch.float32)
+    if M <= 128:
+        assert torch.equal(scales.view(M, K // 128), gs)
+    else:
+        assert torch.equal(scales.view(K // 128, rows_s)[:, :M].t(), gs)
+    # and the split-K / quantization counters are back at zero
+    assert int(ws[:16384].count_nonzero()) == 0
 
 
 # ------------------------------------------------------------------ prefill split-K tail
@@ -249,7 +259,7 @@ import numpy as np, torch
 import fp8_block_scaled_09_b200 as fp8bq, oracle, workloads
 from gpu_util import bf16_to_f64, to_dev_codes, to_dev_f32, tolerance_report
 for i, (M, N, K) in enumerate([(300, 512, 1024), (1000, 768, 2048), (256, 1152, 7168),
-                               (129, 256, 256)]):
+                               (129, 256, 256), (700, 384, 1024), (2100, 640, 512)]):
     x = workloads.activation(M, K, 960 + i, outliers=2)
     qa, sa = oracle.quantize_act(x)
     qw, sw = oracle.quantize_weight(workloads.weight(N, K, 970 + i))
