@@ -782,6 +782,13 @@ def run_profile_case(case: str) -> None:
         gu = torch.randn((4096, 16384), device=dev).mul_(2).to(torch.bfloat16)
         for _ in range(3):
             fp8bq.silu_mul_quantize(gu)
+    elif case == "gateup":
+        # the gate/up GEMM with the SiLU-gated quantization in its epilogue
+        g = W.DRAFTER_GATE_UP
+        qw, sw = fp8bq.quantize_weight(g.make_w().to(dev))
+        qa, sa = fp8bq.quantize_act(g.make_x().to(dev))
+        for _ in range(2):
+            fp8bq.gemm_silu_mul_quantize(qa, sa, qw, sw)
     elif case == "decode-graph":
         # the bench's decode-GEMM step: per-call weight copies, CUDA-graph replays
         xs_host, ws_host = decode_host_inputs()
@@ -821,7 +828,7 @@ def main() -> None:
     ap.add_argument("--quick", action="store_true", help="decode set only (no prefill/workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=("decode", "decode-graph", "midm", "prefill", "quantize",
-                                       "kv", "silu", "nvfp4"),
+                                       "kv", "silu", "gateup", "nvfp4"),
                     help="profiling case: run one kernel family a few times, print a short line")
     args = ap.parse_args()
 

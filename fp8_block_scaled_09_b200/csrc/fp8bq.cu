@@ -22,12 +22,9 @@
 //   gemm_silu_mul_quantize -> M > 128: prefill::gemm_prefill_kernel<256, true>
 //                       (gate/up GEMM whose epilogue quantizes silu(gate) * up);
 //                       smaller M: the decode GEMM, then silu_mul_quantize
-//   linear, M <= 128 -> quantize_act into the workspace, then the decode GEMM,
-//                       which streams its first weight blocks while the
-//                       quantizer still runs (programmatic dependent launch)
-//   linear, M > 128  -> one launch: prefill::gemm_prefill_kernel<256, false, true>
-//                       quantizes X into the workspace while its GEMM consumes
-//                       the finished chunks
+//   linear           -> quantize_act into the workspace, then the gemm path; the
+//                       decode kernel then streams its first weight blocks while
+//                       the quantizer still runs (programmatic dependent launch)
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -122,13 +119,12 @@ EncodeTiledFn encode_fn() {
 
 // Sets the prefill kernel variant's shared-memory limit and checks that it was
 // built with the register count its setmaxnreg split assumes.
-template <bool kSilu, bool kFusedAct>
+template <bool kSilu>
 bool prefill_variant_ready() {
-    auto *k = prefill::gemm_prefill_kernel<kPrefillBN, kSilu, kFusedAct>;
+    auto *k = prefill::gemm_prefill_kernel<kPrefillBN, kSilu>;
     cudaFuncAttributes fa;
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                prefill::Layout<kPrefillBN, kSilu, kFusedAct>::kDynamicSmem) ==
-               cudaSuccess &&
+                                prefill::Layout<kPrefillBN, kSilu>::kDynamicSmem) == cudaSuccess &&
            cudaFuncGetAttributes(&fa, k) == cudaSuccess && fa.numRegs == prefill::kLaunchRegs;
 }
 
@@ -151,9 +147,7 @@ const DeviceInfo *device_info() {
         // the split is only safe if the launch allocates exactly what it was
         // designed for (otherwise setmaxnreg.inc could wait forever).
         cudaFuncAttributes fa;
-        if (!prefill_variant_ready<false, false>() || !prefill_variant_ready<true, false>() ||
-            !prefill_variant_ready<false, true>())
-            return;
+        if (!prefill_variant_ready<false>() || !prefill_variant_ready<true>()) return;
         // CTA-pair prefill kernel: optional; any failure here only leaves it off.
         d.pair_clusters = 0;
         if (pair_prefill_requested() &&
@@ -493,15 +487,7 @@ size_t gemm_ws_bytes_full(int64_t M, int64_t N, int64_t K) {
     return tail ? std::max(need, round256(kPrefillTailBytes)) : need;
 }
 
-// The linear's activation scratch: codes [M, K], then scales.  For M > 128 the
-// scales are stored transposed, [K/128, m_pad] with M rounded up to 128 rows
-// (the single-launch prefill linear reads one 512-byte strip per K chunk).
-int64_t act_scale_rows(int64_t M) {
-    return M > kDecodeMaxM ? (M + prefill::BM - 1) / prefill::BM * prefill::BM : M;
-}
-size_t act_ws_bytes(int64_t M, int64_t K) {
-    return round256(M * K) + round256(act_scale_rows(M) * (K / 128) * 4);
-}
+size_t act_ws_bytes(int64_t M, int64_t K) { return round256(M * K) + round256(M * (K / 128) * 4); }
 
 // The fused linear's workspace holds the GEMM's part first, never shorter than
 // the counter header, then the activation codes and scales (plain scratch).
@@ -610,53 +596,12 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
         float *tail_partials =
             tail_parts ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes)
                        : nullptr;
-        return launch(prefill::gemm_prefill_kernel<kPrefillBN, false, false>, dim3(grid),
-                      dim3(prefill::kNumThreads),
-                      prefill::Layout<kPrefillBN, false, false>::kDynamicSmem, st, ta, tb, sa, sw,
-                      static_cast<__nv_bfloat16 *>(y), static_cast<int>(M), static_cast<int>(N),
-                      static_cast<int>(K), d.status, tail_parts, tail_partials, tail_counters,
-                      prefill::SiluOut{nullptr, nullptr, nullptr}, ta, prefill::FusedAct{});
+        return launch(prefill::gemm_prefill_kernel<kPrefillBN, false>, dim3(grid),
+                      dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN, false>::kDynamicSmem,
+                      st, ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
+                      static_cast<int>(N), static_cast<int>(K), d.status, tail_parts,
+                      tail_partials, tail_counters, prefill::SiluOut{nullptr, nullptr, nullptr});
     }
-}
-
-// Whether the single-launch linear (activation quantization inside the
-// prefill GEMM) takes this shape: its completion counters must fit in the
-// workspace's counter header.
-bool fused_prefill_linear_fits(int64_t M, int64_t K) {
-    const int64_t groups = ((M + prefill::BM - 1) / prefill::BM + prefill::kGroupM - 1) / prefill::kGroupM;
-    return M > kDecodeMaxM && prefill::kActCtrBase + groups * (K / 128) <= prefill::kActClaimSlot;
-}
-
-// The linear layer for M > 128 in one launch: the prefill kernel quantizes X
-// into the workspace (codes qa [M, K], scales transposed saT [K/128, m_pad])
-// while it runs the GEMM on what is done.  ws: the workspace (its counter
-// header at offset 0); part: bytes of its GEMM part.
-cudaError_t launch_linear_prefill(const DeviceInfo &d, const void *x, const uint8_t *qw,
-                                  const float *sw, int64_t M, int64_t N, int64_t K, void *y,
-                                  void *ws, size_t part, uint8_t *qa, float *saT, cudaStream_t st,
-                                  fp8bq_status *err) {
-    *err = FP8BQ_OK;
-    CUtensorMap ta, tb, tx;
-    if (!make_tmap(&ta, qa, M, K, prefill::BM) || !make_tmap(&tb, qw, N, K, kPrefillBN) ||
-        !make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, prefill::BK / 2,
-                      prefill::BM, CU_TENSOR_MAP_SWIZZLE_128B)) {
-        *err = FP8BQ_ERR_CUDA;
-        return cudaSuccess;
-    }
-    const int64_t tiles = ((M + prefill::BM - 1) / prefill::BM) * ((N + kPrefillBN - 1) / kPrefillBN);
-    const int grid = static_cast<int>(tiles < d.sm_count ? tiles : d.sm_count);
-    const int tail_parts = prefill_tail_parts(tiles, grid, K / 128, ws, part);
-    int *ctr = static_cast<int *>(ws);
-    float *tail_partials =
-        tail_parts ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes) : nullptr;
-    const int m_pad = static_cast<int>((M + prefill::BM - 1) / prefill::BM * prefill::BM);
-    return launch(prefill::gemm_prefill_kernel<kPrefillBN, false, true>, dim3(grid),
-                  dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN, false, true>::kDynamicSmem,
-                  st, ta, tb, static_cast<const float *>(saT), sw, static_cast<__nv_bfloat16 *>(y),
-                  static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), d.status, tail_parts,
-                  tail_partials, tail_parts ? ctr : static_cast<int *>(nullptr),
-                  prefill::SiluOut{nullptr, nullptr, nullptr}, tx,
-                  prefill::FusedAct{qa, saT, ctr, m_pad});
 }
 
 // Gate/up GEMM with the SiLU-gated product quantized in its epilogue (M > 128):
@@ -672,12 +617,12 @@ cudaError_t launch_gemm_silu(const DeviceInfo &d, const uint8_t *qa, const float
     }
     const int64_t tiles = ((M + prefill::BM - 1) / prefill::BM) * (I / 128);
     const int grid = static_cast<int>(tiles < d.sm_count ? tiles : d.sm_count);
-    return launch(prefill::gemm_prefill_kernel<kPrefillBN, true, false>, dim3(grid),
-                  dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN, true, false>::kDynamicSmem,
-                  st, ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(nullptr), static_cast<int>(M),
+    return launch(prefill::gemm_prefill_kernel<kPrefillBN, true>, dim3(grid),
+                  dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN, true>::kDynamicSmem, st,
+                  ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(nullptr), static_cast<int>(M),
                   static_cast<int>(2 * I), static_cast<int>(K), d.status, 0,
                   static_cast<float *>(nullptr), static_cast<int *>(nullptr),
-                  prefill::SiluOut{q, s, static_cast<__nv_bfloat16 *>(h)}, ta, prefill::FusedAct{});
+                  prefill::SiluOut{q, s, static_cast<__nv_bfloat16 *>(h)});
 }
 
 // Workspace of the gate/up GEMM with the SiLU epilogue: none on the fused
@@ -953,15 +898,9 @@ fp8bq_status fp8bq_linear(const void *x_bf16, const uint8_t *qw, const float *sw
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint8_t *qa = ws + part;
     float *sa = reinterpret_cast<float *>(qa + round256(M * K));
-    fp8bq_status err;
-    if (fused_prefill_linear_fits(M, K)) {
-        cudaError_t e = launch_linear_prefill(*d, x_bf16, qw, sw, M, N, K, y_bf16, ws, part, qa, sa, s,
-                                              &err);
-        if (err != FP8BQ_OK) return err;
-        return from_cuda(e);
-    }
     cudaError_t e = launch_quantize_act(*d, x_bf16, M, K, qa, sa, s);
     if (e != cudaSuccess) return FP8BQ_ERR_CUDA;
+    fp8bq_status err;
     e = launch_gemm(*d, qa, sa, qw, sw, M, N, K, y_bf16, ws, part, s, &err,
                     /*early_weights=*/true);
     if (err != FP8BQ_OK) return err;

@@ -51,111 +51,29 @@ constexpr int kProducerRegs = 40;    // warpgroup 0 after setmaxnreg.dec
 constexpr int kConsumerRegs = 232;   // warpgroups 1-2 after setmaxnreg.inc
 static_assert(128 * kProducerRegs + 256 * kConsumerRegs <= kNumThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-// With the activation quantizer in warpgroup 0 (kFusedAct), that warpgroup
-// keeps more registers: at 40 its encode loop spilled and ran ~10x slower.
-constexpr int kProducerRegsFused = 72;
-constexpr int kConsumerRegsFused = 216;
-static_assert(128 * kProducerRegsFused + 256 * kConsumerRegsFused <= kNumThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
 constexpr int kFirstPromoWarp = 4;
 constexpr int kPromoWarps = 8;
 constexpr int kGroupM = 16;
 constexpr int kScaleLookahead = 2;   // K chunks of scale prefetch in registers
 
-// Activation quantization inside the GEMM launch (kFusedAct, the linear
-// layer): scale strips of kSaRing chunks in flight, and a two-slot ring of
-// 128 x 128 BF16 activation chunks for the quantizer warp.
-constexpr int kSaRing = 8;
-constexpr int kSaStrip = BM * 4;           // 128 activation scales of one chunk
-constexpr int kQChunkBytes = BM * BK * 2;  // 32 KB of BF16
-constexpr int kQSlots = 2;
-
-template <int BN, bool kSilu = false, bool kFusedAct = false>
+template <int BN, bool kSilu = false>
 struct Layout {
     static_assert(BN == 256, "tile width");
     static constexpr int kA = BM * BK;
     static constexpr int kB = BN * BK;
     static constexpr int kStage = kA + kB;
     static constexpr int kBarOff = kStages * kStage;
-    // full, empty (per stage), tfull, tempty, drain; kFusedAct: sfull, sempty
-    // (per scale strip), qfull (per quantizer slot)
-    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + (kFusedAct ? 2 * kSaRing + kQSlots : 0);
+    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tfull, tempty, drain
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     // SiLU epilogue: per-row group maxima of the two column halves, two tiles
     // deep, each a 64-bit word tagged with the tile's index
     static constexpr int kXchgOff = kMiscOff + 32;
     static constexpr int kXchgBytes = kSilu ? 2 * BM * 2 * 8 : 0;
-    static constexpr int kSaOff = (kXchgOff + kXchgBytes + 1023) & ~1023;
-    static constexpr int kQOff = kSaOff + (kFusedAct ? kSaRing * kSaStrip : 0);
-    static constexpr int kBytes = kQOff + (kFusedAct ? kQSlots * kQChunkBytes : 0);
+    static constexpr int kBytes = kXchgOff + kXchgBytes;
     static constexpr int kDynamicSmem = kBytes + 1024;  // room to align the base to 1024 B
     static_assert(kDynamicSmem <= 227 * 1024, "shared memory");
     static constexpr uint32_t kTmemCols = 2 * BN;
 };
-
-// Header slots (int32, in the counter header at the start of the workspace)
-// used by the in-launch activation quantization: one completion counter per
-// (group of kGroupM m-tiles, K chunk) from kActCtrBase on, the chunk claim
-// counter and the CTA exit counter in the last two slots.  The last CTA to
-// exit zeroes them all again.
-constexpr int kActCtrBase = 64;
-constexpr int kHeaderInts = 4096;
-constexpr int kActClaimSlot = kHeaderInts - 2;
-constexpr int kActExitSlot = kHeaderInts - 1;
-
-struct FusedAct {
-    uint8_t *qa;   // codes [M, K] (workspace)
-    float *saT;    // scales transposed [K/128, m_pad] (workspace)
-    int *ctr;      // the workspace's counter header
-    int m_pad;     // M rounded up to a multiple of 128
-};
-
-// Relaxed (no ordering) load of a global int.
-__device__ __forceinline__ int ld_relaxed_gpu(const int *p) {
-    int v;
-    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Orders this thread's generic-proxy global accesses with its later
-// async-proxy (TMA) accesses.
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Producer side of the in-launch quantization: returns once the activation
-// chunks [0, kb] of an m-tile group are all quantized (counter == gm), reading
-// up to eight counters at once and remembering in `ready_upto` the longest
-// prefix seen complete.  Bounded like every wait.  Acquires on success.
-__device__ __forceinline__ bool wait_act_chunks(const int *ctr, int kb, int KB, int gm,
-                                                int &ready_upto, volatile int *abort,
-                                                int *status) {
-    uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
-        int v[8];
-        const int k0 = ready_upto + 1;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = k0 + j < KB ? ld_relaxed_gpu(ctr + k0 + j) : 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (k0 + j >= KB || v[j] != gm || ready_upto != k0 + j - 1) break;
-            ready_upto = k0 + j;
-        }
-        if (ready_upto >= kb) {
-            __threadfence();  // acquire: the quantizer's stores happen-before what follows
-            return true;
-        }
-        if (it == 0) t0 = global_timer_ns();
-        if ((it & 15u) == 15u) {
-            if (*abort) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-                *abort = 1;
-                atomicExch(status, 6 /* FP8BQ_ERR_TIMEOUT */);
-                return false;
-            }
-        }
-    }
-}
 
 // Split-K tail: when the tiles leave a last wave of at most kTailMaxTiles tiles
 // on the persistent grid, each of those tiles is split K-wise into tail_parts
@@ -331,25 +249,14 @@ struct SiluOut {
     __nv_bfloat16 *h;
 };
 
-// kFusedAct (the linear layer): the A operand is quantized inside the launch.
-// Warp 3 of every CTA claims 128 x 128 chunks of the BF16 activation (tmap_x)
-// in the order the tiles consume them (m-tile group, then K chunk, then m-tile),
-// writes their E4M3 codes to fa.qa and their scales, transposed, to fa.saT, and
-// counts each finished chunk in its (group, K chunk) counter.  The producer
-// waits (bounded) for a chunk's counter before loading its codes, and a
-// 512-byte strip of its scales into a separate ring that the promotion warps
-// read.  No CTA waits for another CTA's progress except through those
-// counters, which any resident CTA's quantizer warp advances, so the grid need
-// not be co-resident.
-template <int BN, bool kSilu, bool kFusedAct>
+template <int BN, bool kSilu>
 __global__ void __launch_bounds__(kNumThreads, 1)
 gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const float *__restrict__ sa,
                     const float *__restrict__ sw, __nv_bfloat16 *__restrict__ y, int M, int N,
                     int K, int *status, int tail_parts, float *tail_partials, int *tail_counters,
-                    SiluOut silu, const __grid_constant__ CUtensorMap tmap_x, FusedAct fa) {
-    static_assert(!(kSilu && kFusedAct), "one variant at a time");
-    using L = Layout<BN, kSilu, kFusedAct>;
+                    SiluOut silu) {
+    using L = Layout<BN, kSilu>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -358,9 +265,6 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     uint64_t *tfull = empty + kStages;
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;
-    uint64_t *sfull = drain + 1;       // kFusedAct: scale strips
-    uint64_t *sempty = sfull + kSaRing;
-    uint64_t *qfull = sempty + kSaRing;  // kFusedAct: quantizer input slots
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
 
@@ -386,13 +290,6 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&tempty[b], kPromoWarps);
         }
         mbar_init(drain, 2);
-        if constexpr (kFusedAct) {
-            for (int i = 0; i < kSaRing; ++i) {
-                mbar_init(&sfull[i], 1);
-                mbar_init(&sempty[i], kPromoWarps);
-            }
-            for (int i = 0; i < kQSlots; ++i) mbar_init(&qfull[i], 1);
-        }
         *abort_flag = 0;
         reinterpret_cast<uint32_t *>(smem + L::kMiscOff + 8)[0] = 0;  // tail verdict
         reinterpret_cast<uint32_t *>(smem + L::kMiscOff + 8)[1] = 0;  // tail arrivals
@@ -406,7 +303,6 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     if (threadIdx.x == 0) {
         prefetch_tmap(&tmap_a);
         prefetch_tmap(&tmap_b);
-        if constexpr (kFusedAct) prefetch_tmap(&tmap_x);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, L::kTmemCols);
@@ -421,8 +317,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     grid_dependency_wait();
 
     if (warp < kFirstPromoWarp) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kFusedAct ? kProducerRegsFused
-                                                                            : kProducerRegs));
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
         if (warp == 0) {
             // ------------------------------------------------------------ TMA producer
             if (lane == 0) {
@@ -430,8 +325,6 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 int64_t issued = 0;
                 bool ok = true;
                 int t, kb0, kb1, part;
-                int cur_g = -1, ready_upto = -1;  // kFusedAct: chunks [0, ready_upto] of group cur_g are done
-                const uint64_t keep = l2_policy_evict_last();
                 for (int w = 0; ok && work_item(w, num_tiles, full_tiles, tail_parts, KB, t, kb0, kb1, part);
                      ++w) {
                     int tm, tn;
@@ -440,34 +333,6 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) {
                             ok = false;
                             break;
-                        }
-                        if constexpr (kFusedAct) {
-                            const int g = tm / kGroupM;
-                            if (g != cur_g) {
-                                cur_g = g;
-                                ready_upto = -1;
-                            }
-                            const int gm = min(kGroupM, m_tiles - g * kGroupM);
-                            if (kb > ready_upto) {
-                                if (!wait_act_chunks(fa.ctr + kActCtrBase + g * KB, kb, KB, gm,
-                                                     ready_upto, abort_flag, status)) {
-                                    ok = false;
-                                    break;
-                                }
-                                // once per newly acquired batch of chunks: the
-                                // TMA loads below read what the acquire made visible
-                                fence_proxy_async_global();
-                            }
-                            const uint32_t si = static_cast<uint32_t>(issued % kSaRing);
-                            const uint32_t sp = static_cast<uint32_t>((issued / kSaRing) & 1);
-                            if (!mbar_wait(&sempty[si], sp ^ 1, abort_flag, status)) {
-                                ok = false;
-                                break;
-                            }
-                            mbar_arrive_expect_tx(&sfull[si], kSaStrip);
-                            bulk_load(smem + L::kSaOff + si * kSaStrip,
-                                      fa.saT + static_cast<int64_t>(kb) * fa.m_pad + tm * BM, kSaStrip,
-                                      &sfull[si], keep);
                         }
                         uint8_t *st = smem + stage * L::kStage;
                         mbar_arrive_expect_tx(&full[stage], L::kStage);
@@ -491,109 +356,6 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 for (int64_t i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
                     mbar_wait(&full[i % kStages], static_cast<uint32_t>((i / kStages) & 1), nullptr,
                               status);
-                if constexpr (kFusedAct)
-                    for (int64_t i = (issued > kSaRing ? issued - kSaRing : 0); i < issued; ++i)
-                        mbar_wait(&sfull[i % kSaRing], static_cast<uint32_t>((i / kSaRing) & 1),
-                                  nullptr, status);
-            }
-        } else if (kFusedAct && warp == 3) {
-            // ------------------------------------------------------------ activation quantizer
-            // Chunk c -> (m-tile group g, K chunk kb, m-tile tm), in the order the
-            // tiles consume them.  Two input slots: the next chunk's load is in
-            // flight while this one is encoded.  A slot holds the chunk's two
-            // 64-channel halves, [128 rows][128 B] each in the 128-byte swizzle
-            // (16-byte unit j of row r at r*128 + 16*(j ^ (r & 7))), so a lane
-            // can own a whole row: lane l encodes rows l, l+32, l+64, l+96, with
-            // no shuffles, and conflict-free shared-memory accesses.  The codes
-            // overwrite the first half in place (a row's unit is read before it
-            // is written) in the same swizzled layout, which one TMA store
-            // writes to the code matrix through the A operand's tensor map.
-            const int64_t n_chunks = static_cast<int64_t>(m_tiles) * KB;
-            const uint64_t stream_once = l2_policy_evict_first();
-            auto claim = [&]() -> int64_t {
-                int c = 0;
-                if (lane == 0) c = atomicAdd(fa.ctr + kActClaimSlot, 1);
-                return __shfl_sync(0xFFFFFFFFu, c, 0);
-            };
-            auto coords = [&](int64_t c, int &g, int &kb, int &tm) {
-                g = static_cast<int>(c / (static_cast<int64_t>(KB) * kGroupM));
-                const int64_t r = c - static_cast<int64_t>(g) * KB * kGroupM;
-                const int gm = min(kGroupM, m_tiles - g * kGroupM);
-                kb = static_cast<int>(r / gm);
-                tm = g * kGroupM + static_cast<int>(r % gm);
-            };
-            auto issue = [&](int64_t c, uint32_t slot) {
-                __syncwarp();  // every lane's reads of the slot come before the load
-                if (lane == 0) {
-                    int g, kb, tm;
-                    coords(c, g, kb, tm);
-                    uint8_t *dst = smem + L::kQOff + slot * kQChunkBytes;
-                    fence_proxy_async_smem();
-                    mbar_arrive_expect_tx(&qfull[slot], kQChunkBytes);
-                    tma_load_2d_hint(dst, &tmap_x, &qfull[slot], kb * BK, tm * BM, stream_once);
-                    tma_load_2d_hint(dst + kQChunkBytes / 2, &tmap_x, &qfull[slot], kb * BK + BK / 2,
-                                     tm * BM, stream_once);
-                }
-            };
-            uint32_t slot = 0, qphase[kQSlots] = {0, 0};
-            int64_t cur = claim();
-            if (cur < n_chunks) issue(cur, 0);
-            while (cur < n_chunks) {
-                const int64_t nxt = claim();
-                if (nxt < n_chunks) issue(nxt, slot ^ 1);
-                bool okw = mbar_wait(&qfull[slot], qphase[slot], abort_flag, status);
-                if (!__all_sync(0xFFFFFFFFu, okw)) {
-                    if (nxt < n_chunks)  // let the load in flight land before the CTA exits
-                        mbar_wait(&qfull[slot ^ 1], qphase[slot ^ 1], nullptr, status);
-                    break;
-                }
-                qphase[slot] ^= 1;
-                int g, kb, tm;
-                coords(cur, g, kb, tm);
-                uint8_t *h0 = smem + L::kQOff + slot * kQChunkBytes;
-                const uint8_t *h1 = h0 + kQChunkBytes / 2;
-                float *st = fa.saT + static_cast<int64_t>(kb) * fa.m_pad + tm * BM;
-                for (int rb = 0; rb < BM / 32; ++rb) {
-                    const int r = rb * 32 + lane;
-                    const int x7 = r & 7;
-                    uint8_t *r0 = h0 + r * 128;
-                    const uint8_t *r1 = h1 + r * 128;
-                    uint32_t m = 0;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        m = max(m, amax_bits8(*reinterpret_cast<const uint4 *>(r0 + ((u ^ x7) << 4))));
-                        m = max(m, amax_bits8(*reinterpret_cast<const uint4 *>(r1 + ((u ^ x7) << 4))));
-                    }
-                    const float scale = scale_from_amax_bits(m);
-                    const float yr = __frcp_rn(scale);
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        // channels 16v .. 16v + 15: units 2v, 2v + 1 of the row
-                        const uint8_t *rs = v < 4 ? r0 : r1;
-                        const int ua = (2 * v) & 7;
-                        const uint4 a = *reinterpret_cast<const uint4 *>(rs + ((ua ^ x7) << 4));
-                        const uint4 b = *reinterpret_cast<const uint4 *>(rs + (((ua + 1) ^ x7) << 4));
-                        const uint2 ca = encode8_y(a, scale, yr);
-                        const uint2 cb = encode8_y(b, scale, yr);
-                        *reinterpret_cast<uint4 *>(r0 + ((v ^ x7) << 4)) = make_uint4(ca.x, ca.y, cb.x, cb.y);
-                    }
-                    st[r] = scale;  // rows past M: scale 1 (zero-filled input)
-                }
-                // The code tile (rows past M are not stored), then the chunk's
-                // counter: the store's writes are complete and ordered before
-                // the release, and before other CTAs' TMA loads of them.
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmap_a, h0, kb * BK, tm * BM);
-                    bulk_commit_group();
-                    bulk_wait_group_all();
-                    fence_proxy_async_global();
-                    __threadfence();
-                    atomicAdd(fa.ctr + kActCtrBase + g * KB + kb, 1);
-                }
-                cur = nxt;
-                slot ^= 1;
             }
         } else if (warp == 1 || warp == 2) {
             // ------------------------------------------------------------ MMA issuers
@@ -635,8 +397,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             }
         }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kFusedAct ? kConsumerRegsFused
-                                                                            : kConsumerRegs));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
         // ------------------------------------------------------------ promotion + epilogue
         const int pw = warp - kFirstPromoWarp;
         const int quarter = warp & 3;  // TMEM lane quarter accessible to this warp
@@ -647,7 +408,6 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
         volatile uint32_t *tail_last = reinterpret_cast<volatile uint32_t *>(smem + L::kMiscOff + 8);
         uint32_t *tail_arrived = reinterpret_cast<uint32_t *>(smem + L::kMiscOff + 12);
         uint32_t buf = 0, bphase = 0;
-        int64_t ci = 0;  // kFusedAct: chunk index over the CTA's work, as the producer counts it
         bool ok = true;
         int t, kb0, kb1, part;
         for (int w = 0; ok && work_item(w, num_tiles, full_tiles, tail_parts, KB, t, kb0, kb1, part);
@@ -672,7 +432,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
             float sa_q[kScaleLookahead], sw_q[kScaleLookahead], swu_q[kScaleLookahead];
 #pragma unroll
             for (int j = 0; j < kScaleLookahead; ++j) {
-                sa_q[j] = (!kFusedAct && row_ok && kb0 + j < kb1) ? __ldg(sa_row + kb0 + j) : 0.0f;
+                sa_q[j] = (row_ok && kb0 + j < kb1) ? __ldg(sa_row + kb0 + j) : 0.0f;
                 sw_q[j] = (col_ok && kb0 + j < kb1) ? __ldg(sw_row + kb0 + j) : 0.0f;
                 if constexpr (kSilu) swu_q[j] = kb0 + j < kb1 ? __ldg(swu_row + kb0 + j) : 0.0f;
             }
@@ -681,25 +441,12 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 for (int j = 0; j < kScaleLookahead; ++j) {
                     const int kb = kbb + j;
                     if (kb >= kb1) break;
-                    float sa_v = sa_q[j];
-                    if constexpr (kFusedAct) {
-                        // this chunk's activation scales, from the strip ring
-                        const uint32_t si = static_cast<uint32_t>(ci % kSaRing);
-                        if (!mbar_wait(&sfull[si], static_cast<uint32_t>((ci / kSaRing) & 1), abort_flag,
-                                       status)) {
-                            ok = false;
-                            break;
-                        }
-                        sa_v = reinterpret_cast<const float *>(smem + L::kSaOff + si * kSaStrip)[row_in_tile];
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sempty[si]);
-                        ++ci;
-                    }
+                    const float sa_v = sa_q[j];
                     const float scale = sa_v * sw_q[j];
                     const float scale1 = kSilu ? sa_v * swu_q[j] : scale;
                     const int kn = kb + kScaleLookahead;
                     if (kn < kb1) {
-                        sa_q[j] = (!kFusedAct && row_ok) ? __ldg(sa_row + kn) : 0.0f;
+                        sa_q[j] = row_ok ? __ldg(sa_row + kn) : 0.0f;
                         sw_q[j] = col_ok ? __ldg(sw_row + kn) : 0.0f;
                         if constexpr (kSilu) swu_q[j] = __ldg(swu_row + kn);
                     }
@@ -864,26 +611,6 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, L::kTmemCols);
-    }
-    if constexpr (kFusedAct) {
-        // The last CTA to get here zeroes the quantization counters (every
-        // other CTA, its quantizer warp included, has finished with them), so
-        // the workspace header is back in its initial state for the next call.
-        volatile int *last = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 16);
-        if (threadIdx.x == 0) {
-            __threadfence();
-            *last = atomicAdd(fa.ctr + kActExitSlot, 1) == static_cast<int>(gridDim.x) - 1;
-        }
-        __syncthreads();
-        if (*last) {
-            __threadfence();
-            const int n = KB * ((m_tiles + kGroupM - 1) / kGroupM);
-            for (int i = threadIdx.x; i < n; i += kNumThreads) fa.ctr[kActCtrBase + i] = 0;
-            if (threadIdx.x == 0) {
-                fa.ctr[kActClaimSlot] = 0;
-                fa.ctr[kActExitSlot] = 0;
-            }
-        }
     }
 }
 

@@ -166,29 +166,6 @@ __device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *m
         : "memory");
 }
 
-// 2-D tile store shared -> global (the map's box and swizzle describe the
-// shared-memory tile), tracked as a bulk async-group of this thread.  Out-of-
-// bounds parts of the box are not written.  x, y >= 0.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x,
-                                             int32_t y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-            reinterpret_cast<uint64_t>(map)),
-        "r"(smem_addr(src)), "r"(x), "r"(y)
-        : "memory");
-}
-
-// Closes this thread's current bulk async-group.
-__device__ __forceinline__ void bulk_commit_group() {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Waits until all of this thread's bulk async-groups are complete (their
-// writes to global memory performed).
-__device__ __forceinline__ void bulk_wait_group_all() {
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 // Untiled bulk copy global -> shared: both addresses 16-byte aligned, `bytes` a
 // multiple of 16; completion counted on `bar`.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,

@@ -123,13 +123,10 @@ FP8BQ_API fp8bq_status fp8bq_quantize_weight(const void *w_bf16, int64_t N, int6
  *       state); calls that share a workspace must be ordered (same stream).
  * Output accuracy: |y - ref| <= 1e-2 |ref| + 2e-3 rms(ref) against the FP64 sum
  * of the dequantized operands; results are deterministic for a given shape.
- * For M <= 16 the call starts reading qw / sw while the previous kernel in the
- * stream may still be running, and lets the next kernel start while its own
- * last blocks finish (programmatic dependent launch), so consecutive calls
- * overlap.  qa, sa and the workspace are read only after the previous kernel
- * has completed.  Reading qw / sw early is safe after this library's weight
- * quantizers, which never let a successor start early; qw / sw must not be
- * written by a foreign kernel that does.
+ * Every operand is read only after the previous kernel in the stream has
+ * completed; the call lets the next kernel launch early (programmatic
+ * dependent launch) and that kernel waits for this one before reading its
+ * output.
  */
 FP8BQ_API fp8bq_status fp8bq_gemm(const uint8_t *qa, const float *sa, const uint8_t *qw, const float *sw,
                         int64_t M, int64_t N, int64_t K, void *y_bf16, void *workspace,

@@ -122,15 +122,15 @@ def test_linear_argument_errors(L):
     assert f(GOOD, GOOD, None, 300, 256, 256, GOOD, GOOD, ws, None) == INVALID
     assert f(ODD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws, None) == MISALIGNED
     # for M > 128: the 16 KB counter header (kept at offset 0 of every
-    # workspace), then the activation codes and scales (transposed, rows padded
-    # to 384), all required (at this K the prefill GEMM has no split-K tail)
+    # workspace), then the activation codes and scales, all required (at this K
+    # the prefill GEMM has no split-K tail to report)
     up = lambda b: -(-b // 256) * 256                # each part padded to 256 bytes
-    assert ws == 16384 + up(300 * 256) + up(384 * 2 * 4)
+    assert ws == 16384 + up(300 * 256) + up(300 * 2 * 4)
     assert f(GOOD, GOOD, GOOD, 300, 256, 256, GOOD, GOOD, ws - 256, None) == WORKSPACE
     # at K >= 16384 the optional tail (header included) replaces the bare header
     ws_long = fp8bq.workspace_size(fp8bq.OP_LINEAR, 300, 256, 16384)
     tail = 16384 + 16 * 4 * 128 * 256 * 4
-    assert ws_long == tail + up(300 * 16384) + up(384 * 128 * 4)
+    assert ws_long == tail + up(300 * 16384) + up(300 * 128 * 4)
     assert f(GOOD, GOOD, GOOD, 300, 256, 16384, GOOD, GOOD, ws_long - tail + 16384 - 256,
              None) == WORKSPACE
     assert f(None, None, None, 0, 256, 256, None, None, 0, None) == OK
@@ -221,8 +221,7 @@ def test_workspace_sizes(L):
     assert lin(8192, 9216, 7168) == 16384 + 8192 * 7168 + 8192 * 56 * 4
     assert lin(16, 9216, 7168) == d + 16 * 7168 + up(16 * 56 * 4)
     assert lin(4096, 7168, 21504) == tail + 4096 * 21504 + 4096 * 168 * 4
-    # M > 128: the scales are kept transposed, [K/128, M rounded up to 128]
-    assert lin(300, 256, 1024) == 16384 + up(300 * 1024) + up(384 * 8 * 4)
+    assert lin(300, 256, 1024) == 16384 + up(300 * 1024) + up(300 * 8 * 4)
     for args in ((1, 128, 128), (17, 384, 1024), (4096, 7168, 21504)):
         assert lin(*args) % 256 == 0 and g(*args) % 256 == 0
     # gate/up with the SiLU epilogue (N = 2I): nothing on the fused prefill path;

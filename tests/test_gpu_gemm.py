@@ -196,20 +196,13 @@ def test_linear_matches_oracle_and_unfused_path(M, N, K):
     y2 = fp8bq.gemm(gq, gs, to_dev_codes(qw), to_dev_f32(sw))
     assert torch.equal(y.t.view(torch.int16), y2.view(torch.int16))
     # the linear's scratch (behind the GEMM's part of a workspace of the
-    # reported size) holds exactly those codes and scales; for M > 128 (one
-    # launch: quantized inside the GEMM) the scales are stored transposed,
-    # [K/128, M rounded up to 128]
+    # reported size) holds exactly those codes and scales
     up = lambda b: -(-b // 256) * 256
-    rows_s = M if M <= 128 else -(-M // 128) * 128
-    off = ws.numel() - up(M * K) - up(rows_s * (K // 128) * 4)
+    off = ws.numel() - up(M * K) - up(M * (K // 128) * 4)
     assert torch.equal(ws[off:off + M * K].view(M, K), gq)
     so = off + up(M * K)
-    scales = ws[so:so + rows_s * (K // 128) * 4].view(torch.float32)
-    if M <= 128:
-        assert torch.equal(scales.view(M, K // 128), gs)
-    else:
-        assert torch.equal(scales.view(K // 128, rows_s)[:, :M].t(), gs)
-    # and the split-K / quantization counters are back at zero
+    assert torch.equal(ws[so:so + M * (K // 128) * 4].view(torch.float32).view(M, K // 128), gs)
+    # and the split-K counters are back at zero
     assert int(ws[:16384].count_nonzero()) == 0
 
 
