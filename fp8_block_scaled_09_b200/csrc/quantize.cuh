@@ -5,8 +5,11 @@
 //
 // Both kernels are bit-exact with the definition: amax of the group/block (an
 // integer max over BF16 magnitude bits, exact for finite values), scale =
-// amax / 448 as an IEEE binary32 division (1.0 when amax is 0), and each code
+// amax / 448 as the IEEE binary32 quotient (1.0 when amax is 0), and each code
 // the saturating round-to-nearest-even E4M3 conversion of fl32(x / scale).
+// Neither division is executed as such: both quotients come from a correctly
+// rounded reciprocal and one FMA correction step (below), which reproduces
+// them on this input domain.
 // The build uses no fast-math and no flush-to-zero, so subnormal scales and
 // quotients follow IEEE arithmetic.
 #pragma once
@@ -22,9 +25,20 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) {
     return __uint_as_float(b16 << 16);
 }
 
+// RN(1 / 448) = 8/7 * 2^-9 rounded to binary32.
+constexpr float kRcp448 = 0x1.24924ap-9f;
+
+// amax / 448, correctly rounded, by the corrected quotient with the constant
+// reciprocal (the method of corrected_quotient below): q = RN(a / 448'),
+// r = a - 448 q exactly, scale = RN(q + r / 448').  Equal to the IEEE quotient
+// for every finite BF16 amax, subnormal results included (checked for all
+// 32639 positive finite values).
 __device__ __forceinline__ float scale_from_amax_bits(uint32_t amax_bits) {
     // amax_bits: BF16 magnitude bits (sign cleared) of the group maximum
-    return amax_bits == 0 ? 1.0f : __fdiv_rn(bf16_bits_to_float(amax_bits), 448.0f);
+    const float a = bf16_bits_to_float(amax_bits);
+    const float q = __fmul_rn(a, kRcp448);
+    const float scale = __fmaf_rn(__fmaf_rn(-q, 448.0f, a), kRcp448, q);
+    return amax_bits == 0 ? 1.0f : scale;
 }
 
 // Smallest scale for which the corrected quotient below reproduces the E4M3
@@ -37,12 +51,14 @@ constexpr float kCorrectedQuotientMinScale = 0x1p-92f;
 // IBM J. Res. Dev. 34(1), 1990; Muller et al., "Handbook of Floating-Point
 // Arithmetic", on division with a fused multiply-add): with q = RN(x y), the
 // residual r = x - q s is exact, and RN(q + r y) is the correctly rounded
-// quotient while no intermediate underflows.  The sign of x is put back so an
-// exact zero keeps it (-0 / s must give the code 0x80).
+// quotient while no intermediate underflows.  The residual is formed negated,
+// n = q s - x = -r, and the result as RN(q - n y): the same value, and for
+// x = -0 (q = -0, n = +0) the sum -0 + -0 keeps the sign, so -0 / s gives the
+// code 0x80 without a separate sign fix-up.
 __device__ __forceinline__ float corrected_quotient(float x, float s, float y) {
     const float q = __fmul_rn(x, y);
-    const float r = __fmaf_rn(-q, s, x);
-    return copysignf(__fmaf_rn(r, y, q), x);
+    const float n = __fmaf_rn(q, s, -x);
+    return __fmaf_rn(-n, y, q);
 }
 
 // Eight BF16 values (one 16-byte vector) -> eight E4M3 codes (8 bytes): each
@@ -86,6 +102,23 @@ __device__ __forceinline__ uint32_t amax_bits8(uint4 v) {
     return m;
 }
 
+// Both halves' magnitude maxima of 16 BF16 values, as two 16-bit lanes
+// (packed per-halfword unsigned max; max_halves() finishes the reduction).
+__device__ __forceinline__ uint32_t amax_bits16_packed(uint4 a, uint4 b) {
+    constexpr uint32_t kMag = 0x7FFF7FFFu;
+    uint32_t m = __vmaxu2(a.x & kMag, a.y & kMag);
+    m = __vmaxu2(m, a.z & kMag);
+    m = __vmaxu2(m, a.w & kMag);
+    m = __vmaxu2(m, b.x & kMag);
+    m = __vmaxu2(m, b.y & kMag);
+    m = __vmaxu2(m, b.z & kMag);
+    return __vmaxu2(m, b.w & kMag);
+}
+
+__device__ __forceinline__ uint32_t max_halves(uint32_t m) {
+    return max(m & 0xFFFFu, m >> 16);
+}
+
 // ------------------------------------------------------------------ activations
 
 // The activation [M, K] is a flat sequence of M K / 128 groups of 256 bytes
@@ -93,8 +126,11 @@ __device__ __forceinline__ uint32_t amax_bits8(uint4 v) {
 // (two per SM) stream chunks of kActChunkGroups groups through a kActStages-deep
 // shared-memory ring with untiled bulk copies, so the bytes in flight do not
 // depend on registers; sixteen consumer warps encode from shared memory, one
-// 16-lane team per group (one 16-byte vector per lane), and store codes and
-// scales straight to global memory.
+// 8-lane team per group, and store codes and scales straight to global
+// memory.  Lane `sub` of a team takes channels [8 sub, 8 sub + 8) and
+// [64 + 8 sub, 64 + 8 sub + 8): each of its two 16-byte loads has the team
+// read 128 contiguous bytes (no bank conflicts), and the per-group work (the
+// shuffles, the scale and its reciprocal) is shared by 16 elements per lane.
 constexpr int kActConsumerWarps = 16;
 constexpr int kActThreads = 32 * (kActConsumerWarps + 1);  // + one producer warp
 constexpr int kActChunkGroups = 64;                         // 16 KB of BF16 per chunk
@@ -153,32 +189,32 @@ quantize_act_kernel(const uint8_t *__restrict__ x, int64_t num_groups, uint2 *__
         }
     } else {
         // ------------------------------------------------------------ consumers
-        const int team = threadIdx.x >> 4;  // 0..31
-        const int sub = threadIdx.x & 15;
+        static_assert(kActChunkGroups == kActConsumerWarps * 4, "one 8-lane team per group");
+        const int gl = threadIdx.x >> 3;  // the team's group within a chunk, 0..63
+        const int sub = threadIdx.x & 7;
         int64_t i = 0;
         for (int64_t c = blockIdx.x; c < num_chunks; c += gridDim.x, ++i) {
             const int s = static_cast<int>(i % kActStages);
             if (!mbar_wait(&full[s], static_cast<uint32_t>((i / kActStages) & 1), abort_flag, status))
                 break;
             const int64_t g0 = c * kActChunkGroups;
-            const uint8_t *st = act_smem + s * kActChunkBytes;
+            const uint8_t *st = act_smem + s * kActChunkBytes + gl * 256 + sub * 16;
+            const bool ok = g0 + gl < num_groups;
+            const uint4 v0 = ok ? *reinterpret_cast<const uint4 *>(st) : make_uint4(0, 0, 0, 0);
+            const uint4 v1 = ok ? *reinterpret_cast<const uint4 *>(st + 128) : make_uint4(0, 0, 0, 0);
+            uint32_t m = amax_bits16_packed(v0, v1);
 #pragma unroll
-            for (int j = 0; j < kActChunkGroups / 32; ++j) {
-                const int gl = team + 32 * j;  // group within the chunk
-                const bool ok = g0 + gl < num_groups;
-                const uint4 v = ok ? *reinterpret_cast<const uint4 *>(st + gl * 256 + sub * 16)
-                                   : make_uint4(0, 0, 0, 0);
-                uint32_t m = amax_bits8(v);
-#pragma unroll
-                for (int off = 8; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-                const float scale = scale_from_amax_bits(m);
-                if (ok) {
-                    q[(g0 + gl) * 16 + sub] = encode8(v, scale);
-                    if (sub == 0) sa[g0 + gl] = scale;
-                }
-            }
+            for (int off = 4; off > 0; off >>= 1) m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+            // every lane has read its vectors: the slot can be refilled
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
+            const float scale = scale_from_amax_bits(max_halves(m));
+            if (ok) {
+                const float y = __frcp_rn(scale);
+                q[(g0 + gl) * 16 + sub] = encode8_y(v0, scale, y);
+                q[(g0 + gl) * 16 + 8 + sub] = encode8_y(v1, scale, y);
+                if (sub == 0) sa[g0 + gl] = scale;
+            }
         }
     }
 }
