@@ -465,3 +465,28 @@ def test_decode_linear_near_ties_matches_unfused():
     torch.cuda.synchronize()
     assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
     check(bf16_to_f64(y), oracle.linear_ref(x, qw, sw))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1024, 7168), (7, 640, 640), (16, 19200, 512), (9, 2048, 2048)])
+def test_decode_linear_special_values_match_unfused(M, N, K):
+    # The decode linear layer (cluster split and stream-K plans) must give an
+    # output bit-identical to quantize_act followed by gemm, also for an
+    # all-zero group (scale 1), BF16 subnormals (scales below 2^-92 take the
+    # IEEE division) and large magnitudes, and within tolerance of the oracle.
+    g = torch.Generator().manual_seed(500 + M)
+    x = torch.randn((M, K), generator=g)
+    x[0, :128] = 0.0
+    x[M - 1, 128:256] *= 1e-39
+    x[M // 2, 256:384] *= 1e30
+    x = x.to(torch.bfloat16)
+    w = workloads.weight(N, K, 600 + M)
+    qw, sw = oracle.quantize_weight(w)
+    xd, qw_d, sw_d = x.cuda(), to_dev_codes(qw), to_dev_f32(sw)
+    ws = fp8bq.new_workspace(fp8bq.OP_LINEAR, M, N, K, "cuda")
+    y = fp8bq.linear(xd, qw_d, sw_d, workspace=ws)
+    qa, sa = fp8bq.quantize_act(xd)
+    y2 = fp8bq.gemm(qa, sa, qw_d, sw_d)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    check(bf16_to_f64(y), oracle.linear_ref(x, qw, sw))
+    assert int(ws[:16384].count_nonzero()) == 0
