@@ -18,7 +18,8 @@
 //   nvfp4_gemm_a16   -> M <= 2: nvfp4::nvfp4_gemv_a16_kernel<1|2> (codes decoded in
 //                       registers, CUDA-core FMA); larger M: nvfp4::nvfp4_gemm_a16_kernel
 //                       (BF16 dequant into shared memory + tcgen05 kind::f16)
-//   silu_mul_quantize-> silu_mul_quantize_kernel (half-warp per 128-channel group)
+//   silu_mul_quantize-> silu_mul_quantize_kernel (half-warp per 128-channel group) or,
+//                       for large problems, silu_mul_quantize_wide_kernel (8-lane teams)
 //   gemm_silu_mul_quantize -> M > 128: prefill::gemm_prefill_kernel<256, true>
 //                       (gate/up GEMM whose epilogue quantizes silu(gate) * up);
 //                       smaller M: the decode GEMM, then silu_mul_quantize
@@ -742,9 +743,22 @@ fp8bq_status fp8bq_silu_mul_quantize(const void *gu_bf16, int64_t M, int64_t I, 
         return FP8BQ_ERR_MISALIGNED;
     const DeviceInfo *d = device_info();
     if (!d) return FP8BQ_ERR_NO_DEVICE;
-    const int64_t groups = M * (I / 128);
+    const int64_t G = I / 128;
+    const int64_t groups = M * G;
+    if (G % 4 == 0 && groups >= static_cast<int64_t>(d->sm_count) * 512) {
+        // large, rows of a multiple of 4 groups: (chunks of a row) x (rows,
+        // strided), about 8 CTAs of 256 threads per SM
+        const int64_t chunks = (G + kSiluWideGroupsPerCta - 1) / kSiluWideGroupsPerCta;
+        const int64_t rows = std::max<int64_t>(
+            1, std::min<int64_t>(M, (static_cast<int64_t>(d->sm_count) * 8 + chunks - 1) / chunks));
+        return from_cuda(launch(silu_mul_quantize_wide_kernel,
+                                dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(rows)),
+                                dim3(kSiluThreads), 0, static_cast<cudaStream_t>(stream),
+                                static_cast<const uint4 *>(gu_bf16), M, I,
+                                reinterpret_cast<uint2 *>(q_e4m3), s, static_cast<uint4 *>(h_bf16)));
+    }
     const int64_t warps = (groups + 1) / 2;
-    const int64_t blocks = std::min<int64_t>((warps + kSiluThreads / 32 - 1) / (kSiluThreads / 32),
+    const int64_t blocks = std::min<int64_t>((warps + kSiluWarps - 1) / kSiluWarps,
                                              static_cast<int64_t>(d->sm_count) * 16);
     return from_cuda(launch(silu_mul_quantize_kernel, dim3(static_cast<unsigned>(blocks)),
                             dim3(kSiluThreads), 0, static_cast<cudaStream_t>(stream),

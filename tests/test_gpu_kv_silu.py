@@ -138,8 +138,12 @@ def _within_one_bf16_step(got_bits, exact):
     return same, same | neighbour | zeros
 
 
+# (700, 5248): 41 groups per row (not a multiple of 4).  (2000, 5120): large
+# enough for the 8-lane-team kernel, 40 groups per row so the second 32-group
+# chunk of a row is ragged (some warps of its CTA have no group), and more rows
+# than the grid's row count
 @pytest.mark.parametrize("M,I,scale", [(1, 128, 1.0), (3, 384, 4.0), (130, 8192, 2.0),
-                                        (17, 1024, 30.0)])
+                                        (17, 1024, 30.0), (700, 5248, 1.0), (2000, 5120, 1.0)])
 def test_silu_mul_quantize_matches_oracle(M, I, scale):
     rng = np.random.default_rng(M * 7 + I)
     gu = torch.from_numpy(rng.standard_normal((M, 2 * I)).astype(np.float32) * scale).to(torch.bfloat16)
