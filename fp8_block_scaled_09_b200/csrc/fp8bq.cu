@@ -121,12 +121,28 @@ EncodeTiledFn encode_fn() {
 // Sets the prefill kernel variant's shared-memory limit and checks that it was
 // built with the register count its setmaxnreg split assumes.
 template <bool kSilu>
-bool prefill_variant_ready() {
-    auto *k = prefill::gemm_prefill_kernel<kPrefillBN, kSilu>;
+bool prefill_instance_ready(void (*k)(CUtensorMap, CUtensorMap, const float *, const float *,
+                                      __nv_bfloat16 *, int, int, int, int *, int, float *, int *,
+                                      prefill::SiluOut)) {
     cudaFuncAttributes fa;
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 prefill::Layout<kPrefillBN, kSilu>::kDynamicSmem) == cudaSuccess &&
            cudaFuncGetAttributes(&fa, k) == cudaSuccess && fa.numRegs == prefill::kLaunchRegs;
+}
+
+// The prefill kernel instance for a K (raster group of prefill::group_m(K/128)
+// m-tiles).
+template <bool kSilu>
+auto prefill_kernel_for(int64_t K) {
+    return prefill::group_m(static_cast<int>(K / 128)) == 32
+               ? prefill::gemm_prefill_kernel<kPrefillBN, kSilu, 32>
+               : prefill::gemm_prefill_kernel<kPrefillBN, kSilu, 16>;
+}
+
+template <bool kSilu>
+bool prefill_variant_ready() {
+    return prefill_instance_ready<kSilu>(prefill::gemm_prefill_kernel<kPrefillBN, kSilu, 16>) &&
+           prefill_instance_ready<kSilu>(prefill::gemm_prefill_kernel<kPrefillBN, kSilu, 32>);
 }
 
 // Current device's info, set up once per device (kernel attributes, status word).
@@ -597,7 +613,7 @@ cudaError_t launch_gemm(const DeviceInfo &d, const uint8_t *qa, const float *sa,
         float *tail_partials =
             tail_parts ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + decode::kCounterBytes)
                        : nullptr;
-        return launch(prefill::gemm_prefill_kernel<kPrefillBN, false>, dim3(grid),
+        return launch(prefill_kernel_for<false>(K), dim3(grid),
                       dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN, false>::kDynamicSmem,
                       st, ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(y), static_cast<int>(M),
                       static_cast<int>(N), static_cast<int>(K), d.status, tail_parts,
@@ -618,7 +634,7 @@ cudaError_t launch_gemm_silu(const DeviceInfo &d, const uint8_t *qa, const float
     }
     const int64_t tiles = ((M + prefill::BM - 1) / prefill::BM) * (I / 128);
     const int grid = static_cast<int>(tiles < d.sm_count ? tiles : d.sm_count);
-    return launch(prefill::gemm_prefill_kernel<kPrefillBN, true>, dim3(grid),
+    return launch(prefill_kernel_for<true>(K), dim3(grid),
                   dim3(prefill::kNumThreads), prefill::Layout<kPrefillBN, true>::kDynamicSmem, st,
                   ta, tb, sa, sw, static_cast<__nv_bfloat16 *>(nullptr), static_cast<int>(M),
                   static_cast<int>(2 * I), static_cast<int>(K), d.status, 0,

@@ -26,8 +26,8 @@
 //               128-column weight block, whose scale is a single sw per chunk.
 // Register budget: launched at 168 per thread (384 x 168 = 64512); after the
 // split 128 x 40 + 256 x 232 = 64512, the same total.
-// Tiles are walked in groups of kGroupM m-tiles so the tiles resident at one
-// time share A and B rows in L2.
+// Tiles are walked in groups of group_m(K) m-tiles (m fastest within a group)
+// so the tiles resident at one time share A and B rows in L2.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -53,7 +53,15 @@ static_assert(128 * kProducerRegs + 256 * kConsumerRegs <= kNumThreads * kLaunch
               "register split exceeds the launch allocation");
 constexpr int kFirstPromoWarp = 4;
 constexpr int kPromoWarps = 8;
-constexpr int kGroupM = 16;
+// m-tiles per raster group: each group streams every weight tile once, so
+// larger groups re-read the weights less often (QKV 8192 x 9216 x 7168: 322 MB
+// of DRAM reads with 16, 204 MB with 32, for 125 MB of operands), as long as
+// the group's A rows (group x 128 x K bytes) leave L2 room for the weight tiles
+// in flight: 32 up to K = 10240, i.e. KB = K / 128 <= 80 (at most 42 MB of A),
+// 16 beyond (64 m-tiles, all of A, raised the reads instead).  A template
+// parameter of the kernel (a run-time group size costs the 40-register
+// producer warp a spill).
+__host__ __device__ constexpr int group_m(int KB) { return KB <= 80 ? 32 : 16; }
 constexpr int kScaleLookahead = 2;   // K chunks of scale prefetch in registers
 
 template <int BN, bool kSilu = false>
@@ -106,11 +114,12 @@ __device__ __forceinline__ bool work_item(int w, int num_tiles, int full_tiles, 
     return true;
 }
 
-__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int &tm, int &tn) {
-    const int group = kGroupM * n_tiles;
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int group_rows, int &tm,
+                                            int &tn) {
+    const int group = group_rows * n_tiles;
     const int g = t / group, r = t - g * group;
-    const int first_m = g * kGroupM;
-    const int gm = min(kGroupM, m_tiles - first_m);
+    const int first_m = g * group_rows;
+    const int gm = min(group_rows, m_tiles - first_m);
     tm = first_m + r % gm;
     tn = r / gm;
 }
@@ -249,7 +258,7 @@ struct SiluOut {
     __nv_bfloat16 *h;
 };
 
-template <int BN, bool kSilu>
+template <int BN, bool kSilu, int kGroupRows>
 __global__ void __launch_bounds__(kNumThreads, 1)
 gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const float *__restrict__ sa,
@@ -328,7 +337,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 for (int w = 0; ok && work_item(w, num_tiles, full_tiles, tail_parts, KB, t, kb0, kb1, part);
                      ++w) {
                     int tm, tn;
-                    tile_coords(t, m_tiles, n_tiles, tm, tn);
+                    tile_coords(t, m_tiles, n_tiles, kGroupRows, tm, tn);
                     for (int kb = kb0; kb < kb1; ++kb) {
                         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) {
                             ok = false;
@@ -413,7 +422,7 @@ gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
         for (int w = 0; ok && work_item(w, num_tiles, full_tiles, tail_parts, KB, t, kb0, kb1, part);
              ++w) {
             int tm, tn;
-            tile_coords(t, m_tiles, n_tiles, tm, tn);
+            tile_coords(t, m_tiles, n_tiles, kGroupRows, tm, tn);
             const int grow = tm * BM + row_in_tile;
             // plain: this thread's 128 output columns, one weight block; SiLU:
             // 64 gate and the same 64 up channels, two weight blocks
