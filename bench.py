@@ -582,7 +582,7 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
         "roofline": {"bound": "tensor", "achieved": pq["gemm_tflops"], "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": pq["gemm_tflops"] / fp8_peak,
                      "frac_of_sustained": pq["gemm_tflops"] / fp8_peak_sus, "traffic": None,
-                     "kernel": "fp8bq::prefill::gemm_prefill_kernel<256>",
+                     "kernel": "fp8bq::prefill::gemm_prefill_kernel<256, false, 32>",
                      "peak_source": f"{peaks['source']} cuBLAS BF16 x 2 (nominal FP8/BF16 ratio)"},
         "timing": f"mean of {iters} graph replays, CUDA events, L2 flushed (256 MB write + read) before each",
     }

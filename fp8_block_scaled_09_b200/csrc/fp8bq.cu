@@ -11,8 +11,8 @@
 //                       64 or 128; each n-block split over a cluster of CTAs
 //                       reduced in shared memory, or stream-K over all weight
 //                       blocks with a global split-K reduction)
-//   gemm, M > 128    -> prefill::gemm_prefill_kernel<256> (persistent tcgen05;
-//                       the CTA-pair kernel prefill2 is built but not dispatched)
+//   gemm, M > 128    -> prefill::gemm_prefill_kernel<256, false, 16|32> (persistent tcgen05;
+//                       the CTA-pair kernel prefill2 only with FP8BQ_PREFILL_PAIRS=1)
 //   kv_write_e4m3    -> kv_write_e4m3_kernel (warp per K/V row, slot scatter)
 //   nvfp4_quantize_weight -> nvfp4 amax, quantize and global-scale kernels
 //   nvfp4_gemm_a16   -> M <= 2: nvfp4::nvfp4_gemv_a16_kernel<1|2> (codes decoded in
@@ -20,7 +20,7 @@
 //                       (BF16 dequant into shared memory + tcgen05 kind::f16)
 //   silu_mul_quantize-> silu_mul_quantize_kernel (half-warp per 128-channel group) or,
 //                       for large problems, silu_mul_quantize_wide_kernel (8-lane teams)
-//   gemm_silu_mul_quantize -> M > 128: prefill::gemm_prefill_kernel<256, true>
+//   gemm_silu_mul_quantize -> M > 128: prefill::gemm_prefill_kernel<256, true, 16|32>
 //                       (gate/up GEMM whose epilogue quantizes silu(gate) * up);
 //                       smaller M: the decode GEMM, then silu_mul_quantize
 //   linear           -> quantize_act into the workspace, then the gemm path; the
