@@ -60,11 +60,11 @@ STEP_VARIANTS = 2            # steps alternate between copies 0-2 and 3-5
 # launch), measured by ncu on `bench.py --only decode-graph`.  Valid only for the decode
 # kernel source it was taken on: `kernel_sha` is the SHA-256 (first 16 hex digits) of
 # gemm_decode.cuh + ptx.cuh; when the source differs, the traffic is reported as null.
-DECODE_TRAFFIC = {"bytes_per_launch": 57736917, "kernel_sha": "fdeb213142315536",
+DECODE_TRAFFIC = {"bytes_per_launch": 57746954, "kernel_sha": "bf3c4541ec7aa1fd",
                   "how": "ncu --cache-control none --clock-control none --metrics "
                          "dram__bytes_read.sum,dram__bytes_write.sum on the 24 graph-replayed "
                          "decode GEMM launches (4 steps of 6) of `bench.py --only decode-graph`: "
-                         "57.31 MB read + 0.43 MB written per launch"}
+                         "57.30 MB read + 0.44 MB written per launch"}
 DECODE_WORKLOAD = ("decode GEMV set: fp8bq_linear, M in {1,4,8} x {fused QKV W[9216,7168], "
                    "o_proj W[7168,7168]}, E4M3 128x128-blocked weights, X BF16 N(0,1) with "
                    "7 outlier channels x20")
