@@ -53,6 +53,10 @@ import workloads as W  # noqa: E402
 
 METRIC = "FP8 block-scaled GEMM TFLOPS (prefill) & HBM GB/s (decode), % of roofline, 1 B200"
 FP8_OVER_BF16 = 2.0          # nominal dense ratio 4.5 / 2.25 PFLOP/s
+# Nominal B200 figures, for the second fraction reported beside the measured
+# one: HBM3e 7.7 TB/s (HGX), dense FP8 4.5 PFLOP/s.
+NOMINAL_HBM_GBS = 7700.0
+NOMINAL_FP8_TFLOPS = 4500.0
 COPIES = 6                   # device copies of each decode weight (3 calls per shape per step)
 STEP_VARIANTS = 2            # steps alternate between copies 0-2 and 3-5
 # DRAM bytes (read + write) per decode GEMM launch, averaged over consecutive launches of the
@@ -418,7 +422,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     sha = decode_kernel_sha()
     traffic = DECODE_TRAFFIC["bytes_per_launch"] if DECODE_TRAFFIC["kernel_sha"] == sha else None
     roofline = {"bound": "hbm", "achieved": gemm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                "frac": gemm_gbs / peaks["hbm_gbs"], "frac_of_nominal": gemm_gbs / NOMINAL_HBM_GBS,
+                "traffic": traffic,
                 "traffic_source": DECODE_TRAFFIC["how"] if traffic is not None else
                                   f"null: no capture for this decode kernel source ({sha})",
                 "kernel": "fp8bq::decode::gemm_decode_kernel<16> (cluster split)",
@@ -581,7 +586,8 @@ def prefill_and_workloads(torch, fp8bq, dev, clocks, peaks, fp8_peak, fp8_peak_s
         "gemm_us": pq["gemm_us"], "cpu_baseline": pq.get("cpu_baseline"),
         "roofline": {"bound": "tensor", "achieved": pq["gemm_tflops"], "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": pq["gemm_tflops"] / fp8_peak,
-                     "frac_of_sustained": pq["gemm_tflops"] / fp8_peak_sus, "traffic": None,
+                     "frac_of_sustained": pq["gemm_tflops"] / fp8_peak_sus,
+                     "frac_of_nominal": pq["gemm_tflops"] / NOMINAL_FP8_TFLOPS, "traffic": None,
                      "kernel": "fp8bq::prefill::gemm_prefill_kernel<256, false, 32>",
                      "peak_source": f"{peaks['source']} cuBLAS BF16 x 2 (nominal FP8/BF16 ratio)"},
         "timing": f"mean of {iters} graph replays, CUDA events, L2 flushed (256 MB write + read) before each",
