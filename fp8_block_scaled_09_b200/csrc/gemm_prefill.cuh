@@ -156,25 +156,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // acc[0..63] from TMEM columns taddr0 .. taddr0 + 63 with scale0, acc[64..127]
 // from taddr1 .. taddr1 + 63 with scale1 (for a plain tile, taddr1 = taddr0 +
 // 64 and scale1 = scale0).  The TMEM loads go in two batches of 64 columns,
-// one wait each: the second batch is in flight while the FMAs of the first
-// run, and it is returned in `last` after its wait, so the caller releases
-// the TMEM buffer after two load waits (not four) and finishes those 64 FMAs
-// afterwards (measured +3% on every prefill shape over four 32-column loads
-// with a wait each).  Loads and waits live in one asm statement so no
-// register is read before its wait.
+// one 32x32b.x64 load and one wait each: the second batch is in flight while
+// the FMAs of the first run, and it is returned in `last` after its wait, so
+// the caller releases the TMEM buffer after two load waits (not four) and
+// finishes those 64 FMAs afterwards (measured +3% on every prefill shape over
+// four 32-column loads with a wait each; one .x64 load per batch instead of
+// two .x32 gained another 0.7-1% on QKV, fc and long o_proj).  Loads and waits
+// live in one asm statement so no register is read before its wait.
 __device__ __forceinline__ void promote_chunk(uint32_t taddr0, uint32_t taddr1, float scale0,
                                               float scale1, float (&acc)[128], float (&last)[64]) {
     asm volatile(
         "{\n\t"
         ".reg .f32 ra<32>, rb<32>;\n\t"
-        ".reg .b32 ta1, ta3;\n\t"
-        "add.u32 ta1, %129, 32;\n\t"
-        "add.u32 ta3, %131, 32;\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {ra0,ra1,ra2,ra3,ra4,ra5,ra6,ra7,ra8,ra9,ra10,ra11,ra12,ra13,ra14,ra15,ra16,ra17,ra18,ra19,ra20,ra21,ra22,ra23,ra24,ra25,ra26,ra27,ra28,ra29,ra30,ra31}, [%129];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {rb0,rb1,rb2,rb3,rb4,rb5,rb6,rb7,rb8,rb9,rb10,rb11,rb12,rb13,rb14,rb15,rb16,rb17,rb18,rb19,rb20,rb21,rb22,rb23,rb24,rb25,rb26,rb27,rb28,rb29,rb30,rb31}, [ta1];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {ra0,ra1,ra2,ra3,ra4,ra5,ra6,ra7,ra8,ra9,ra10,ra11,ra12,ra13,ra14,ra15,ra16,ra17,ra18,ra19,ra20,ra21,ra22,ra23,ra24,ra25,ra26,ra27,ra28,ra29,ra30,ra31,rb0,rb1,rb2,rb3,rb4,rb5,rb6,rb7,rb8,rb9,rb10,rb11,rb12,rb13,rb14,rb15,rb16,rb17,rb18,rb19,rb20,rb21,rb22,rb23,rb24,rb25,rb26,rb27,rb28,rb29,rb30,rb31}, [%129];\n\t"
         "tcgen05.wait::ld.sync.aligned;\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%131];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [ta3];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131];\n\t"
         "fma.rn.f32 %0, ra0, %128, %0;\n\t"
         "fma.rn.f32 %1, ra1, %128, %1;\n\t"
         "fma.rn.f32 %2, ra2, %128, %2;\n\t"
